@@ -1,0 +1,397 @@
+// api.cu -- the C ABI declared in include/dust.h: host-side validation,
+// workspace layout, and the sequence of launches for each entry point.
+// Nothing here allocates or synchronises (except dust_poll_status, which
+// exists to read the device status word back).
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+dust_status fail(dust_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+dust_status ok() { return DUST_OK; }
+
+dust_status cuda_status(cudaError_t e, const char* where) {
+    if (e == cudaSuccess) return DUST_OK;
+    return fail(DUST_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+#define DUST_REQUIRE(cond, code, ...)                 \
+    do {                                               \
+        if (!(cond)) return fail(code, __VA_ARGS__);   \
+    } while (0)
+
+#define DUST_TRY(expr)                                 \
+    do {                                               \
+        dust_status _s = (expr);                       \
+        if (_s != DUST_OK) return _s;                  \
+    } while (0)
+
+dust_status check_noise(const dust_noise& nz) {
+    DUST_REQUIRE(nz.draw_count > 0, DUST_ERR_INVALID_ARG, "draw_count must be > 0");
+    DUST_REQUIRE(nz.K_total > 0, DUST_ERR_INVALID_ARG, "K_total must be > 0");
+    DUST_REQUIRE(std::isfinite(nz.sigma) && nz.sigma > 0.0f, DUST_ERR_INVALID_ARG, "sigma must be finite and > 0");
+    DUST_REQUIRE(static_cast<uint64_t>(nz.draw_begin) + nz.draw_count <= (1ull << 32), DUST_ERR_INVALID_ARG,
+                 "draw_begin + draw_count exceeds 2^32");
+    return ok();
+}
+
+dust_status check_ptr(const void* p, const char* name, bool nullable = false) {
+    if (p == nullptr) {
+        DUST_REQUIRE(nullable, DUST_ERR_INVALID_ARG, "%s must not be NULL", name);
+        return ok();
+    }
+    DUST_REQUIRE(aligned(p, 16), DUST_ERR_ALIGNMENT, "%s is not 16-byte aligned", name);
+    return ok();
+}
+
+dust_status check_seq(const int32_t* offs, int n_seq, int K, int T) {
+    DUST_TRY(check_ptr(offs, "seq_offsets"));
+    DUST_REQUIRE(n_seq >= 1, DUST_ERR_INVALID_ARG, "n_seq must be >= 1");
+    DUST_REQUIRE(static_cast<long long>(K) * n_seq < (1ll << 31), DUST_ERR_INVALID_ARG,
+                 "draws x sequences must be < 2^31");
+    (void)T;
+    return ok();
+}
+
+// Workspace: [status (256 B)][region 0][region 1]...; every region 256-byte aligned.
+struct Layout {
+    size_t off = dust::kStatusBytes;
+    size_t add(size_t bytes) {
+        const size_t o = off;
+        off = dust::align_up(off + bytes, 256);
+        return o;
+    }
+};
+
+uint8_t* region(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
+
+size_t dtype_bytes(dust_dtype dt) { return dt == DUST_BF16 ? 2 : 4; }
+
+// ---- GEMM dispatch shared by weight_grad, logits and head_step ----------------
+struct GemmPlan {
+    bool tc = false;
+    int splits = 1;
+    size_t partial_bytes = 0;
+};
+
+GemmPlan plan_gemm(int M, int N, int K, dust_dtype dt, bool a_kmajor, bool b_kmajor) {
+    GemmPlan p;
+    p.tc = dt == DUST_BF16 && dust::gemm_tc_supported(M, N, K, a_kmajor, b_kmajor);
+    p.splits = p.tc ? dust::gemm_tc_splits(M, N, K) : dust::gemm_simt_splits(M, N, K);
+    p.partial_bytes = p.splits > 1 ? sizeof(float) * static_cast<size_t>(p.splits) * M * N : 0;
+    return p;
+}
+
+dust_status run_gemm(const GemmPlan& p, const void* A, bool ak, int lda, const void* B, bool bk, int ldb,
+                     dust_dtype dt, int M, int N, int K, float* C, int ldc, int accumulate, float* partial,
+                     uint32_t* status, cudaStream_t st) {
+    cudaError_t e = p.tc ? dust::launch_gemm_tc(A, ak, lda, B, bk, ldb, M, N, K, C, ldc, accumulate, partial,
+                                                p.splits, status, st)
+                         : dust::launch_gemm_simt(A, ak, lda, B, bk, ldb, dt, M, N, K, C, ldc, accumulate,
+                                                  partial, p.splits, st);
+    return cuda_status(e, p.tc ? "tcgen05 GEMM" : "CUDA-core GEMM");
+}
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+}  // namespace
+
+extern "C" {
+
+const char* dust_status_string(dust_status s) {
+    switch (s) {
+        case DUST_OK: return "DUST_OK";
+        case DUST_ERR_INVALID_ARG: return "DUST_ERR_INVALID_ARG";
+        case DUST_ERR_UNSUPPORTED: return "DUST_ERR_UNSUPPORTED";
+        case DUST_ERR_ALIGNMENT: return "DUST_ERR_ALIGNMENT";
+        case DUST_ERR_WORKSPACE: return "DUST_ERR_WORKSPACE";
+        case DUST_ERR_CUDA: return "DUST_ERR_CUDA";
+        case DUST_ERR_TIMEOUT: return "DUST_ERR_TIMEOUT";
+    }
+    return "DUST_ERR_UNKNOWN";
+}
+
+const char* dust_last_error(void) { return g_last_error.c_str(); }
+
+int dust_abi_version(void) { return DUST_ABI_VERSION; }
+
+dust_status dust_check_offsets(const int32_t* offs, int n_seq, int T) {
+    DUST_REQUIRE(offs != nullptr, DUST_ERR_INVALID_ARG, "seq_offsets must not be NULL");
+    DUST_REQUIRE(n_seq >= 1, DUST_ERR_INVALID_ARG, "n_seq must be >= 1");
+    DUST_REQUIRE(offs[0] == 0, DUST_ERR_INVALID_ARG, "seq_offsets[0] must be 0 (got %d)", offs[0]);
+    for (int q = 0; q < n_seq; ++q)
+        DUST_REQUIRE(offs[q + 1] >= offs[q], DUST_ERR_INVALID_ARG, "seq_offsets decrease at %d", q);
+    DUST_REQUIRE(offs[n_seq] == T, DUST_ERR_INVALID_ARG, "seq_offsets[n_seq] = %d, expected T = %d",
+                 offs[n_seq], T);
+    return ok();
+}
+
+dust_status dust_poll_status(void* ws, void* stream) {
+    DUST_REQUIRE(ws != nullptr, DUST_ERR_INVALID_ARG, "ws must not be NULL");
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof word, cudaMemcpyDeviceToHost, as_stream(stream));
+    if (e == cudaSuccess) e = cudaStreamSynchronize(as_stream(stream));
+    DUST_TRY(cuda_status(e, "dust_poll_status"));
+    if (word == 0) return ok();
+    DUST_TRY(cuda_status(cudaMemsetAsync(ws, 0, sizeof word, as_stream(stream)), "dust_poll_status"));
+    return fail(DUST_ERR_TIMEOUT, "a kernel's bounded wait ran out (status word 0x%08x)", word);
+}
+
+// ------------------------------------------------------------------ a4
+dust_status dust_reward_scan(const float* c, float* r, int K, int T, const int32_t* seq_offsets, int n_seq,
+                             float gamma, void* stream) {
+    DUST_REQUIRE(K > 0 && T > 0, DUST_ERR_INVALID_ARG, "K and T must be > 0 (K=%d, T=%d)", K, T);
+    DUST_REQUIRE(std::isfinite(gamma) && gamma >= 0.0f && gamma <= 1.0f, DUST_ERR_INVALID_ARG,
+                 "gamma must be in [0, 1]");
+    DUST_TRY(check_ptr(c, "c"));
+    DUST_TRY(check_ptr(r, "r"));
+    DUST_TRY(check_seq(seq_offsets, n_seq, K, T));
+    return cuda_status(dust::launch_reward_scan(c, r, K, T, seq_offsets, n_seq, gamma, as_stream(stream)),
+                       "dust_reward_scan");
+}
+
+// ------------------------------------------------------------------ a5
+size_t dust_layer_estimate_workspace(int draw_count, int T, int d_out, int is_r, float gamma) {
+    (void)d_out;
+    Layout L;
+    if (!is_r && gamma != 0.0f && draw_count > 0 && T > 0) L.add(sizeof(float) * static_cast<size_t>(draw_count) * T);
+    return L.off;
+}
+
+dust_status dust_layer_estimate(const float* c_or_r, int is_r, int T, int d_out, const int32_t* seq_offsets,
+                                int n_seq, float gamma, dust_noise nz, float* g_hat, void* g_hat_bf16,
+                                int accumulate, void* ws, size_t ws_bytes, void* stream) {
+    DUST_TRY(check_noise(nz));
+    DUST_REQUIRE(T > 0 && d_out > 0, DUST_ERR_INVALID_ARG, "T and d_out must be > 0 (T=%d, d_out=%d)", T, d_out);
+    DUST_REQUIRE(std::isfinite(gamma) && gamma >= 0.0f && gamma <= 1.0f, DUST_ERR_INVALID_ARG,
+                 "gamma must be in [0, 1]");
+    DUST_TRY(check_ptr(c_or_r, "c_or_r"));
+    DUST_TRY(check_ptr(g_hat, "g_hat"));
+    DUST_TRY(check_ptr(g_hat_bf16, "g_hat_bf16", true));
+    const bool need_scan = !is_r && gamma != 0.0f;
+    if (need_scan) DUST_TRY(check_seq(seq_offsets, n_seq, static_cast<int>(nz.draw_count), T));
+    const size_t need = dust_layer_estimate_workspace(static_cast<int>(nz.draw_count), T, d_out, is_r, gamma);
+    // ws may be NULL when no scan is needed (the estimate itself uses no scratch)
+    DUST_TRY(check_ptr(ws, "ws", need <= dust::kStatusBytes));
+    DUST_REQUIRE(ws == nullptr || ws_bytes >= need, DUST_ERR_WORKSPACE, "workspace %zu bytes < %zu", ws_bytes, need);
+    cudaStream_t st = as_stream(stream);
+    const float* r = c_or_r;
+    if (need_scan) {
+        float* rw = reinterpret_cast<float*>(region(ws, dust::kStatusBytes));
+        DUST_TRY(cuda_status(dust::launch_reward_scan(c_or_r, rw, static_cast<int>(nz.draw_count), T, seq_offsets,
+                                                      n_seq, gamma, st),
+                             "dust_layer_estimate (scan)"));
+        r = rw;
+    }
+    return cuda_status(dust::launch_layer_estimate(r, T, d_out, nz, g_hat, g_hat_bf16, accumulate, st),
+                       "dust_layer_estimate");
+}
+
+// ------------------------------------------------------------------ a6
+static GemmPlan weight_grad_plan(int T, int d_in, int d_out, dust_dtype dt) {
+    // C[d_out][d_in] = sum_t g[t][o] X[t][i]: A = g (M-major), B = X (N-major)
+    return plan_gemm(d_out, d_in, T, dt, false, false);
+}
+
+size_t dust_weight_grad_workspace(int T, int d_in, int d_out, dust_dtype dt) {
+    Layout L;
+    if (T > 0 && d_in > 0 && d_out > 0) L.add(weight_grad_plan(T, d_in, d_out, dt).partial_bytes);
+    return L.off;
+}
+
+dust_status dust_weight_grad(const void* g_hat, const void* X, dust_dtype dt, int T, int d_in, int d_out,
+                             float* G_W, int accumulate, void* ws, size_t ws_bytes, void* stream) {
+    DUST_REQUIRE(dt == DUST_F32 || dt == DUST_BF16, DUST_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
+    DUST_REQUIRE(T > 0 && d_in > 0 && d_out > 0, DUST_ERR_INVALID_ARG, "T, d_in, d_out must be > 0");
+    DUST_TRY(check_ptr(g_hat, "g_hat"));
+    DUST_TRY(check_ptr(X, "X"));
+    DUST_TRY(check_ptr(G_W, "G_W"));
+    DUST_TRY(check_ptr(ws, "ws"));
+    const size_t need = dust_weight_grad_workspace(T, d_in, d_out, dt);
+    DUST_REQUIRE(ws_bytes >= need, DUST_ERR_WORKSPACE, "workspace %zu bytes < %zu", ws_bytes, need);
+    const GemmPlan p = weight_grad_plan(T, d_in, d_out, dt);
+    float* partial = reinterpret_cast<float*>(region(ws, dust::kStatusBytes));
+    return run_gemm(p, g_hat, false, d_out, X, false, d_in, dt, d_out, d_in, T, G_W, d_in, accumulate, partial,
+                    static_cast<uint32_t*>(ws), as_stream(stream));
+}
+
+// ------------------------------------------------------------------ a2
+static GemmPlan logits_plan(int T, int d_in, int V, dust_dtype dt) {
+    // Z[T][V] = sum_k X[t][k] W[v][k]: A = X (K-major), B = W (K-major)
+    return plan_gemm(T, V, d_in, dt, true, true);
+}
+
+size_t dust_logits_workspace(int T, int d_in, int V, dust_dtype dt) {
+    Layout L;
+    if (T > 0 && d_in > 0 && V > 0) L.add(logits_plan(T, d_in, V, dt).partial_bytes);
+    return L.off;
+}
+
+dust_status dust_logits(const void* X, const void* W, dust_dtype dt, int T, int d_in, int V, float* Z, void* ws,
+                        size_t ws_bytes, void* stream) {
+    DUST_REQUIRE(dt == DUST_F32 || dt == DUST_BF16, DUST_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
+    DUST_REQUIRE(T > 0 && d_in > 0 && V > 0, DUST_ERR_INVALID_ARG, "T, d_in, V must be > 0");
+    DUST_TRY(check_ptr(X, "X"));
+    DUST_TRY(check_ptr(W, "W"));
+    DUST_TRY(check_ptr(Z, "Z"));
+    DUST_TRY(check_ptr(ws, "ws"));
+    const size_t need = dust_logits_workspace(T, d_in, V, dt);
+    DUST_REQUIRE(ws_bytes >= need, DUST_ERR_WORKSPACE, "workspace %zu bytes < %zu", ws_bytes, need);
+    const GemmPlan p = logits_plan(T, d_in, V, dt);
+    return run_gemm(p, X, true, d_in, W, true, d_in, dt, T, V, d_in, Z, V, 0,
+                    reinterpret_cast<float*>(region(ws, dust::kStatusBytes)), static_cast<uint32_t*>(ws),
+                    as_stream(stream));
+}
+
+dust_status dust_head_row_stats(const float* Z, const int32_t* targets, int T, int V, float* lse, float* ell,
+                                void* stream) {
+    DUST_REQUIRE(T > 0 && V > 0, DUST_ERR_INVALID_ARG, "T and V must be > 0");
+    DUST_TRY(check_ptr(Z, "Z"));
+    DUST_TRY(check_ptr(targets, "targets"));
+    DUST_TRY(check_ptr(lse, "lse"));
+    DUST_TRY(check_ptr(ell, "ell", true));
+    return cuda_status(dust::launch_row_stats(Z, targets, T, V, lse, ell, as_stream(stream)), "dust_head_row_stats");
+}
+
+// ------------------------------------------------------------------ head step
+namespace {
+struct HeadLayout {
+    size_t z = 0, lse = 0, g16 = 0, zpart = 0, wpart = 0, total = 0;
+    GemmPlan zplan, wplan;
+};
+
+HeadLayout head_layout(int T, int d_in, int V, dust_dtype dt, int has_Z, int want_G_W) {
+    HeadLayout h;
+    Layout L;
+    if (!has_Z) {
+        h.zplan = logits_plan(T, d_in, V, dt);
+        h.z = L.add(sizeof(float) * static_cast<size_t>(T) * V);
+        h.zpart = L.add(h.zplan.partial_bytes);
+    }
+    h.lse = L.add(sizeof(float) * static_cast<size_t>(T));
+    if (want_G_W) {
+        h.wplan = weight_grad_plan(T, d_in, V, dt);
+        if (dt == DUST_BF16) h.g16 = L.add(sizeof(uint16_t) * static_cast<size_t>(T) * V);
+        h.wpart = L.add(h.wplan.partial_bytes);
+    }
+    h.total = L.off;
+    return h;
+}
+}  // namespace
+
+size_t dust_head_step_workspace(int T, int d_in, int V, dust_dtype dt, int has_Z, int want_G_W) {
+    if (T <= 0 || V <= 0 || ((!has_Z || want_G_W) && d_in <= 0)) return dust::kStatusBytes;
+    return head_layout(T, d_in, V, dt, has_Z, want_G_W).total;
+}
+
+dust_status dust_head_step(const void* X, const void* W, dust_dtype dt, const float* Z, const int32_t* targets, int T,
+                           int d_in, int V, int Vc, dust_noise nz, float* c_out, float* g_hat, void* g_hat_bf16,
+                           float* G_W, int accumulate, void* ws, size_t ws_bytes, void* stream) {
+    DUST_TRY(check_noise(nz));
+    DUST_REQUIRE(dt == DUST_F32 || dt == DUST_BF16, DUST_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
+    DUST_REQUIRE(T > 0 && V > 0, DUST_ERR_INVALID_ARG, "T and V must be > 0");
+    DUST_REQUIRE(Vc > 0 && V % Vc == 0, DUST_ERR_INVALID_ARG, "Vc=%d must divide V=%d", Vc, V);
+    DUST_REQUIRE(Vc % 128 == 0 && Vc <= 1024, DUST_ERR_UNSUPPORTED,
+                 "Vc=%d unsupported (a multiple of 128, at most 1024)", Vc);
+    DUST_REQUIRE(V / Vc <= 65535, DUST_ERR_INVALID_ARG, "too many chunks");
+    const bool has_Z = Z != nullptr, want_G_W = G_W != nullptr;
+    if (!has_Z || want_G_W) {
+        DUST_REQUIRE(d_in > 0, DUST_ERR_INVALID_ARG, "d_in must be > 0");
+        DUST_TRY(check_ptr(X, "X"));
+    }
+    if (!has_Z) DUST_TRY(check_ptr(W, "W"));
+    DUST_TRY(check_ptr(Z, "Z", true));
+    DUST_TRY(check_ptr(targets, "targets"));
+    DUST_TRY(check_ptr(c_out, "c_out", true));
+    DUST_TRY(check_ptr(g_hat, "g_hat"));
+    DUST_TRY(check_ptr(g_hat_bf16, "g_hat_bf16", true));
+    DUST_TRY(check_ptr(G_W, "G_W", true));
+    DUST_TRY(check_ptr(ws, "ws"));
+    const HeadLayout h = head_layout(T, d_in, V, dt, has_Z, want_G_W);
+    DUST_REQUIRE(ws_bytes >= h.total, DUST_ERR_WORKSPACE, "workspace %zu bytes < %zu", ws_bytes, h.total);
+    cudaStream_t st = as_stream(stream);
+    uint32_t* status = static_cast<uint32_t*>(ws);
+
+    const float* Zuse = Z;
+    if (!has_Z) {   // a2: clean logits into the workspace
+        float* Zw = reinterpret_cast<float*>(region(ws, h.z));
+        DUST_TRY(run_gemm(h.zplan, X, true, d_in, W, true, d_in, dt, T, V, d_in, Zw, V, 0,
+                          reinterpret_cast<float*>(region(ws, h.zpart)), status, st));
+        Zuse = Zw;
+    }
+    float* lse = reinterpret_cast<float*>(region(ws, h.lse));
+    DUST_TRY(cuda_status(dust::launch_row_stats(Zuse, targets, T, V, lse, nullptr, st), "dust_head_step (row stats)"));
+    void* g16 = g_hat_bf16;
+    if (want_G_W && dt == DUST_BF16 && g16 == nullptr) g16 = region(ws, h.g16);
+    DUST_TRY(cuda_status(dust::launch_head_chunks(Zuse, lse, targets, T, V, Vc, nz, c_out, g_hat, g16, accumulate, st),
+                         "dust_head_step (chunks)"));
+    if (!want_G_W) return ok();
+    const void* gA = dt == DUST_BF16 ? g16 : static_cast<const void*>(g_hat);
+    return run_gemm(h.wplan, gA, false, V, X, false, d_in, dt, V, d_in, T, G_W, d_in, 0,
+                    reinterpret_cast<float*>(region(ws, h.wpart)), status, st);
+}
+
+// ------------------------------------------------------------------ harness
+dust_status dust_noise_fill(dust_noise nz, uint32_t stream_id, int t0, int n_tok, int j0, int n_ch, float* out,
+                            void* stream) {
+    DUST_REQUIRE(nz.draw_count > 0, DUST_ERR_INVALID_ARG, "draw_count must be > 0");
+    DUST_REQUIRE(t0 >= 0 && n_tok > 0 && j0 >= 0 && n_ch > 0, DUST_ERR_INVALID_ARG, "bad token/channel range");
+    DUST_TRY(check_ptr(out, "out"));
+    return cuda_status(dust::launch_noise_fill(nz, stream_id, t0, n_tok, j0, n_ch, out, as_stream(stream)),
+                       "dust_noise_fill");
+}
+
+dust_status dust_synth_costs(const float* u, int T, int d_out, dust_noise nz, float eps_scale, float* c, void* stream) {
+    DUST_REQUIRE(nz.draw_count > 0, DUST_ERR_INVALID_ARG, "draw_count must be > 0");
+    DUST_REQUIRE(std::isfinite(nz.sigma) && nz.sigma >= 0.0f, DUST_ERR_INVALID_ARG, "sigma must be finite and >= 0");
+    DUST_REQUIRE(std::isfinite(eps_scale), DUST_ERR_INVALID_ARG, "eps_scale must be finite");
+    DUST_REQUIRE(T > 0 && d_out > 0, DUST_ERR_INVALID_ARG, "T and d_out must be > 0");
+    DUST_TRY(check_ptr(u, "u"));
+    DUST_TRY(check_ptr(c, "c"));
+    return cuda_status(dust::launch_synth_costs(u, T, d_out, nz, eps_scale, c, as_stream(stream)), "dust_synth_costs");
+}
+
+size_t dust_toy_suffix_workspace(int draw_count, int T, int d, int dh, int V) {
+    if (draw_count <= 0 || T <= 0 || d <= 0 || dh <= 0 || V <= 0) return dust::kStatusBytes;
+    return dust::toy_suffix_workspace_bytes(draw_count, T, d, dh, V);
+}
+
+dust_status dust_toy_suffix_losses(const float* Y, int T, int d, const int32_t* seq_offsets, int n_seq, const float* Wq,
+                                   const float* Wk, const float* Wv, const float* Wo, int dh, const float* Wout, int V,
+                                   const int32_t* targets, dust_noise nz, float* loss, float* c, void* ws,
+                                   size_t ws_bytes, void* stream) {
+    DUST_TRY(check_noise(nz));
+    DUST_REQUIRE(T > 0 && d > 0 && dh > 0 && V > 0, DUST_ERR_INVALID_ARG, "T, d, dh, V must be > 0");
+    DUST_REQUIRE(d % 4 == 0 && d <= 1024 && dh <= 128, DUST_ERR_UNSUPPORTED,
+                 "toy suffix supports d %% 4 == 0, d <= 1024, dh <= 128");
+    DUST_TRY(check_seq(seq_offsets, n_seq, 1, T));
+    const void* ptrs[] = {Y, Wq, Wk, Wv, Wo, Wout, targets, loss, ws};
+    const char* names[] = {"Y", "Wq", "Wk", "Wv", "Wo", "Wout", "targets", "loss", "ws"};
+    for (int i = 0; i < 9; ++i) DUST_TRY(check_ptr(ptrs[i], names[i]));
+    DUST_TRY(check_ptr(c, "c", true));
+    const size_t need = dust_toy_suffix_workspace(static_cast<int>(nz.draw_count), T, d, dh, V);
+    DUST_REQUIRE(ws_bytes >= need, DUST_ERR_WORKSPACE, "workspace %zu bytes < %zu", ws_bytes, need);
+    return cuda_status(dust::run_toy_suffix(Y, T, d, seq_offsets, n_seq, Wq, Wk, Wv, Wo, dh, Wout, V, targets, nz, loss,
+                                            c, ws, as_stream(stream)),
+                       "dust_toy_suffix_losses");
+}
+
+}  // extern "C"

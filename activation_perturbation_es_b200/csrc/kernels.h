@@ -1,0 +1,68 @@
+// kernels.h -- internal launchers (one per kernel family).  Each enqueues on
+// `stream` and returns the launch status; argument validation happens in
+// api.cu before any of these is called.
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "dust.h"
+
+namespace dust {
+
+// a4 (reward_scan.cu)
+cudaError_t launch_reward_scan(const float* c, float* r, int K, int T, const int32_t* offs,
+                               int n_seq, float gamma, cudaStream_t stream);
+
+// a1 + a5 (layer_estimate.cu): g (+)= scale * sum_k r[k][t] a(draw_begin + k, t, j)
+cudaError_t launch_layer_estimate(const float* r, int T, int d_out, const dust_noise& nz,
+                                  float* g, void* g_bf16, int accumulate, cudaStream_t stream);
+
+// a1 harness (noise_fill.cu)
+cudaError_t launch_noise_fill(const dust_noise& nz, uint32_t stream_id, int t0, int n_tok, int j0,
+                              int n_ch, float* out, cudaStream_t stream);
+cudaError_t launch_synth_costs(const float* u, int T, int d_out, const dust_noise& nz,
+                               float eps_scale, float* c, cudaStream_t stream);
+
+// a6 / a2 on CUDA cores (gemm_simt.cu):
+//   C[m][n] = sum_k A(m, k) B(k, n), C row-major [M][N] with leading dim ldc.
+//   A(m, k) = a_kmajor ? A[m * lda + k] : A[k * lda + m]
+//   B(k, n) = b_kmajor ? B[n * ldb + k] : B[k * ldb + n]
+// Split over k into `splits` slices; slice s writes partial[s][M][N] (fp32)
+// unless splits == 1, in which case it writes (or adds to, accumulate) C.
+cudaError_t launch_gemm_simt(const void* A, bool a_kmajor, int lda, const void* B, bool b_kmajor,
+                             int ldb, dust_dtype dt, int M, int N, int K, float* C, int ldc,
+                             int accumulate, float* partial, int splits, cudaStream_t stream);
+int gemm_simt_splits(int M, int N, int K);
+// C (+)= sum_s partial[s]  (fixed order), C [M][N] leading dim ldc
+cudaError_t launch_splitk_reduce(const float* partial, int splits, int M, int N, float* C, int ldc,
+                                 int accumulate, cudaStream_t stream);
+
+// a6 / a2 on tcgen05 tensor cores (gemm_tcgen05.cu), bf16 operands, fp32 out.
+// Same contract as launch_gemm_simt; returns cudaErrorNotSupported when the
+// shape is outside what the kernel handles (multiples of 16 in M, N).
+cudaError_t launch_gemm_tc(const void* A, bool a_kmajor, int lda, const void* B, bool b_kmajor,
+                           int ldb, int M, int N, int K, float* C, int ldc, int accumulate,
+                           float* partial, int splits, uint32_t* status, cudaStream_t stream);
+int gemm_tc_splits(int M, int N, int K);
+bool gemm_tc_supported(int M, int N, int K, bool a_kmajor, bool b_kmajor);
+
+// a2 row statistics + a3/a5 fused head (head.cu)
+cudaError_t launch_row_stats(const float* Z, const int32_t* targets, int T, int V, float* lse,
+                             float* ell, cudaStream_t stream);
+cudaError_t launch_head_chunks(const float* Z, const float* lse, const int32_t* targets, int T,
+                               int V, int Vc, const dust_noise& nz, float* c_out, float* g,
+                               void* g_bf16, int accumulate, cudaStream_t stream);
+
+// harness: toy causal suffix (toy_suffix.cu)
+size_t toy_suffix_workspace_bytes(int draw_count, int T, int d, int dh, int V);
+cudaError_t run_toy_suffix(const float* Y, int T, int d, const int32_t* offs, int n_seq, const float* Wq,
+                           const float* Wk, const float* Wv, const float* Wo, int dh, const float* Wout, int V,
+                           const int32_t* targets, const dust_noise& nz, float* loss, float* c, void* ws,
+                           cudaStream_t st);
+
+// fp32 -> bf16 (RNE) copy
+cudaError_t launch_to_bf16(const float* src, void* dst, size_t n, cudaStream_t stream);
+
+}  // namespace dust

@@ -1,0 +1,107 @@
+// layer_estimate.cu -- a1 + a5: noise regeneration and the noise-weighted
+// reduction over draws.
+//
+// cnblogs Dust explainer, section "信用分配：一次前向，两种奖励", error
+// equation: g_t = -(1/(K sigma)) sum_i r_t^(i) a_t^(i).
+//
+// Design (B200): the work is K x T x d_out Gaussians, each regenerated from its
+// coordinates (noise.cuh) and consumed by one FMA; nothing K x T x d is ever
+// stored, and the only HBM traffic is r (4 bytes per draw x token, a warp-wide
+// broadcast) and g (written once).  The kernel is therefore bound by the SM
+// issue rate, not by HBM.  One thread owns (token t, channel quad q): a single
+// Philox call per draw yields its 4 channels, so the counter words that do not
+// depend on the draw (first-round product of the quad, key schedule) are
+// hoisted out of the draw loop.  Two draws per iteration give the scheduler two
+// independent Philox chains.  Blocks are 256 threads: quads along x (coalesced
+// 128-bit stores of g), tokens along y.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "noise.cuh"
+
+namespace dust {
+
+namespace {
+
+__device__ __forceinline__ void fma4(float4& acc, float r, const float4& a) {
+    acc.x = __fmaf_rn(r, a.x, acc.x);
+    acc.y = __fmaf_rn(r, a.y, acc.y);
+    acc.z = __fmaf_rn(r, a.z, acc.z);
+    acc.w = __fmaf_rn(r, a.w, acc.w);
+}
+
+__global__ void __launch_bounds__(256)
+layer_estimate_kernel(const float* __restrict__ r, int T, int d_out, int nq, uint32_t seed,
+                      uint32_t layer, uint32_t draw_begin, int nd, float scale,
+                      float* __restrict__ g, __nv_bfloat16* __restrict__ g16, int accumulate) {
+    const int q = blockIdx.x * blockDim.x + threadIdx.x;
+    if (q >= nq) return;
+    const bool vec_ok = (d_out & 3) == 0;
+    for (int t = blockIdx.y * blockDim.y + threadIdx.y; t < T; t += gridDim.y * blockDim.y) {
+        float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 acc1 = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float* rt = r + t;
+        int k = 0;
+        for (; k + 2 <= nd; k += 2) {
+            const float r0 = __ldg(rt + static_cast<size_t>(k) * T);
+            const float r1 = __ldg(rt + static_cast<size_t>(k + 1) * T);
+            const float4 a0 = gauss4(seed, layer, draw_begin + k, t, q, 0);
+            const float4 a1 = gauss4(seed, layer, draw_begin + k + 1, t, q, 0);
+            fma4(acc0, r0, a0);
+            fma4(acc1, r1, a1);
+        }
+        if (k < nd) {
+            const float r0 = __ldg(rt + static_cast<size_t>(k) * T);
+            fma4(acc0, r0, gauss4(seed, layer, draw_begin + k, t, q, 0));
+        }
+        float4 out = make_float4((acc0.x + acc1.x) * scale, (acc0.y + acc1.y) * scale,
+                                 (acc0.z + acc1.z) * scale, (acc0.w + acc1.w) * scale);
+        const size_t base = static_cast<size_t>(t) * d_out + 4 * static_cast<size_t>(q);
+        if (vec_ok) {
+            float4* gp = reinterpret_cast<float4*>(g + base);
+            if (accumulate) {
+                const float4 o = *gp;
+                out.x += o.x; out.y += o.y; out.z += o.z; out.w += o.w;
+            }
+            *gp = out;
+            if (g16) {
+                __nv_bfloat162 lo = __floats2bfloat162_rn(out.x, out.y);
+                __nv_bfloat162 hi = __floats2bfloat162_rn(out.z, out.w);
+                uint2 pk;
+                pk.x = *reinterpret_cast<uint32_t*>(&lo);
+                pk.y = *reinterpret_cast<uint32_t*>(&hi);
+                *reinterpret_cast<uint2*>(g16 + base) = pk;
+            }
+        } else {
+            const float v[4] = {out.x, out.y, out.z, out.w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                if (4 * q + w >= d_out) break;
+                float x = v[w];
+                if (accumulate) x += g[base + w];
+                g[base + w] = x;
+                if (g16) g16[base + w] = __float2bfloat16_rn(x);
+            }
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_layer_estimate(const float* r, int T, int d_out, const dust_noise& nz, float* g,
+                                  void* g_bf16, int accumulate, cudaStream_t stream) {
+    const int nq = (d_out + 3) / 4;
+    int bx = nq >= 128 ? 128 : ((nq + 31) / 32) * 32;
+    const int by = 256 / bx;
+    const unsigned gx = static_cast<unsigned>(ceil_div(nq, bx));
+    const long long ty = ceil_div(T, by);
+    const unsigned gy = static_cast<unsigned>(ty < 65535 ? ty : 65535);
+    const float scale = static_cast<float>(-1.0 / (static_cast<double>(nz.K_total) * nz.sigma));
+    layer_estimate_kernel<<<dim3(gx, gy), dim3(bx, by), 0, stream>>>(
+        r, T, d_out, nq, nz.seed, nz.layer, nz.draw_begin, static_cast<int>(nz.draw_count), scale, g,
+        static_cast<__nv_bfloat16*>(g_bf16), accumulate);
+    return cudaGetLastError();
+}
+
+}  // namespace dust

@@ -1,0 +1,289 @@
+"""Python binding of libdust.so (the C ABI in include/dust.h).
+
+Argument marshalling only: tensors must be CUDA tensors of the documented
+dtype and layout; this module turns them into pointers and the current torch
+stream, allocates the caller-owned outputs and workspace with torch, and calls
+the library.  Every step of the estimator runs in the library's kernels; there
+is no CPU or PyTorch fallback, and a missing library raises.
+
+Names follow the C ABI with the ``dust_`` prefix dropped.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libdust.so")
+
+F32, BF16 = 0, 1
+STATUS = {0: "DUST_OK", 1: "DUST_ERR_INVALID_ARG", 2: "DUST_ERR_UNSUPPORTED", 3: "DUST_ERR_ALIGNMENT",
+          4: "DUST_ERR_WORKSPACE", 5: "DUST_ERR_CUDA", 6: "DUST_ERR_TIMEOUT"}
+
+
+class DustError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class _Noise(C.Structure):
+    _fields_ = [("seed", C.c_uint32), ("layer", C.c_uint32), ("draw_begin", C.c_uint32),
+                ("draw_count", C.c_uint32), ("K_total", C.c_uint32), ("sigma", C.c_float)]
+
+
+@dataclass(frozen=True)
+class Noise:
+    """Which draws of which layer a call handles (dust_noise)."""
+    seed: int
+    layer: int
+    draw_begin: int
+    draw_count: int
+    K_total: int
+    sigma: float
+
+    def c(self) -> _Noise:
+        return _Noise(self.seed, self.layer, self.draw_begin, self.draw_count, self.K_total, self.sigma)
+
+
+_lib = None
+_vp, _sz, _i, _f, _u = C.c_void_p, C.c_size_t, C.c_int, C.c_float, C.c_uint32
+
+_SIGS = {
+    "dust_status_string": ([_i], C.c_char_p),
+    "dust_last_error": ([], C.c_char_p),
+    "dust_abi_version": ([], _i),
+    "dust_check_offsets": ([_vp, _i, _i], _i),
+    "dust_poll_status": ([_vp, _vp], _i),
+    "dust_reward_scan": ([_vp, _vp, _i, _i, _vp, _i, _f, _vp], _i),
+    "dust_layer_estimate": ([_vp, _i, _i, _i, _vp, _i, _f, _Noise, _vp, _vp, _i, _vp, _sz, _vp], _i),
+    "dust_layer_estimate_workspace": ([_i, _i, _i, _i, _f], _sz),
+    "dust_weight_grad": ([_vp, _vp, _i, _i, _i, _i, _vp, _i, _vp, _sz, _vp], _i),
+    "dust_weight_grad_workspace": ([_i, _i, _i, _i], _sz),
+    "dust_logits": ([_vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp], _i),
+    "dust_logits_workspace": ([_i, _i, _i, _i], _sz),
+    "dust_head_row_stats": ([_vp, _vp, _i, _i, _vp, _vp, _vp], _i),
+    "dust_head_step": ([_vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _Noise, _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp], _i),
+    "dust_head_step_workspace": ([_i, _i, _i, _i, _i, _i], _sz),
+    "dust_noise_fill": ([_Noise, _u, _i, _i, _i, _i, _vp, _vp], _i),
+    "dust_synth_costs": ([_vp, _i, _i, _Noise, _f, _vp, _vp], _i),
+    "dust_toy_suffix_losses": ([_vp, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp, _Noise, _vp, _vp,
+                                _vp, _sz, _vp], _i),
+    "dust_toy_suffix_workspace": ([_i, _i, _i, _i, _i], _sz),
+}
+
+
+def lib() -> C.CDLL:
+    """Load libdust.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m activation_perturbation_es_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise DustError(status, lib().dust_last_error().decode())
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _opt(t, name, dtype=None):
+    return None if t is None else _dev(t, name, dtype)
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise ValueError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+_ws = {}
+
+
+def workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A cached caller-owned workspace of at least nbytes on the current device."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    cur = _ws.get(dev)
+    if cur is None or cur.numel() < nbytes:
+        cur = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=dev)
+        _ws[dev] = cur
+    return cur
+
+
+def check_offsets(seq_offsets, T: int) -> None:
+    """Validate sequence offsets on the host (numpy / CPU tensor / list)."""
+    off = np.ascontiguousarray(np.asarray(seq_offsets.cpu() if isinstance(seq_offsets, torch.Tensor)
+                                          else seq_offsets), dtype=np.int32)
+    _check(lib().dust_check_offsets(off.ctypes.data, len(off) - 1, T))
+
+
+def poll_status(ws: torch.Tensor) -> None:
+    _check(lib().dust_poll_status(_dev(ws, "ws"), _stream()))
+
+
+# ------------------------------------------------------------------ a4
+def reward_scan(c: torch.Tensor, seq_offsets: torch.Tensor, gamma: float, out: torch.Tensor | None = None):
+    K, T = c.shape
+    r = torch.empty_like(c) if out is None else out
+    _check(lib().dust_reward_scan(_dev(c, "c", torch.float32), _dev(r, "r", torch.float32), K, T,
+                                  _dev(seq_offsets, "seq_offsets", torch.int32), seq_offsets.numel() - 1,
+                                  float(gamma), _stream()))
+    return r
+
+
+# ------------------------------------------------------------------ a5
+def layer_estimate(c_or_r: torch.Tensor, is_r: bool, seq_offsets, gamma: float, noise: Noise, d_out: int,
+                   g_hat: torch.Tensor | None = None, g_hat_bf16: torch.Tensor | bool | None = None,
+                   accumulate: bool = False):
+    """Returns (g_hat [T][d_out] fp32, g_hat_bf16 or None)."""
+    nd, T = c_or_r.shape
+    if nd != noise.draw_count:
+        raise ValueError("c_or_r must have draw_count rows")
+    dev = c_or_r.device
+    if g_hat is None:
+        g_hat = torch.empty(T, d_out, dtype=torch.float32, device=dev)
+    if g_hat_bf16 is True:
+        g_hat_bf16 = torch.empty(T, d_out, dtype=torch.bfloat16, device=dev)
+    elif g_hat_bf16 is False:
+        g_hat_bf16 = None
+    need = lib().dust_layer_estimate_workspace(nd, T, d_out, int(bool(is_r)), float(gamma))
+    ws = workspace(need, dev)
+    offs = None if seq_offsets is None else _dev(seq_offsets, "seq_offsets", torch.int32)
+    n_seq = 1 if seq_offsets is None else seq_offsets.numel() - 1
+    _check(lib().dust_layer_estimate(_dev(c_or_r, "c_or_r", torch.float32), int(bool(is_r)), T, d_out, offs, n_seq,
+                                     float(gamma), noise.c(), _dev(g_hat, "g_hat", torch.float32),
+                                     _opt(g_hat_bf16, "g_hat_bf16", torch.bfloat16), int(bool(accumulate)),
+                                     ws.data_ptr(), ws.numel(), _stream()))
+    return g_hat, g_hat_bf16
+
+
+# ------------------------------------------------------------------ a6
+def weight_grad(g_hat: torch.Tensor, X: torch.Tensor, G_W: torch.Tensor | None = None, accumulate: bool = False):
+    T, d_out = g_hat.shape
+    d_in = X.shape[1]
+    if X.shape[0] != T or X.dtype != g_hat.dtype:
+        raise ValueError("g_hat and X must share T and dtype")
+    dt = _dtype_code(X)
+    if G_W is None:
+        G_W = torch.empty(d_out, d_in, dtype=torch.float32, device=X.device)
+    ws = workspace(lib().dust_weight_grad_workspace(T, d_in, d_out, dt), X.device)
+    _check(lib().dust_weight_grad(_dev(g_hat, "g_hat"), _dev(X, "X"), dt, T, d_in, d_out,
+                                  _dev(G_W, "G_W", torch.float32), int(bool(accumulate)), ws.data_ptr(),
+                                  ws.numel(), _stream()))
+    return G_W
+
+
+# ------------------------------------------------------------------ a2
+def logits(X: torch.Tensor, W: torch.Tensor, Z: torch.Tensor | None = None):
+    T, d_in = X.shape
+    V = W.shape[0]
+    dt = _dtype_code(X)
+    if W.dtype != X.dtype or W.shape[1] != d_in:
+        raise ValueError("X and W must share d_in and dtype")
+    if Z is None:
+        Z = torch.empty(T, V, dtype=torch.float32, device=X.device)
+    ws = workspace(lib().dust_logits_workspace(T, d_in, V, dt), X.device)
+    _check(lib().dust_logits(_dev(X, "X"), _dev(W, "W"), dt, T, d_in, V, _dev(Z, "Z", torch.float32),
+                             ws.data_ptr(), ws.numel(), _stream()))
+    return Z
+
+
+def head_row_stats(Z: torch.Tensor, targets: torch.Tensor):
+    T, V = Z.shape
+    lse = torch.empty(T, dtype=torch.float32, device=Z.device)
+    ell = torch.empty(T, dtype=torch.float32, device=Z.device)
+    _check(lib().dust_head_row_stats(_dev(Z, "Z", torch.float32), _dev(targets, "targets", torch.int32), T, V,
+                                     lse.data_ptr(), ell.data_ptr(), _stream()))
+    return lse, ell
+
+
+# ------------------------------------------------------------------ head step
+def head_step(targets: torch.Tensor, Vc: int, noise: Noise, *, Z: torch.Tensor | None = None,
+              X: torch.Tensor | None = None, W: torch.Tensor | None = None, V: int | None = None,
+              want_c: bool = False, want_bf16: bool = False, want_G_W: bool = False,
+              g_hat: torch.Tensor | None = None, g_hat_bf16: torch.Tensor | None = None,
+              accumulate: bool = False):
+    """Returns dict with g_hat, and c / g_hat_bf16 / G_W when requested."""
+    T = targets.numel()
+    dev = targets.device
+    if Z is not None:
+        V = Z.shape[1]
+    elif W is not None:
+        V = W.shape[0]
+    if V is None:
+        raise ValueError("need Z or W")
+    ref = X if X is not None else W
+    dt = _dtype_code(ref) if ref is not None else F32
+    d_in = X.shape[1] if X is not None else (W.shape[1] if W is not None else 0)
+    if g_hat is None:
+        g_hat = torch.empty(T, V, dtype=torch.float32, device=dev)
+    c = torch.empty(V // Vc, noise.draw_count, T, dtype=torch.float32, device=dev) if want_c else None
+    g16 = g_hat_bf16
+    if g16 is None and want_bf16:
+        g16 = torch.empty(T, V, dtype=torch.bfloat16, device=dev)
+    G_W = torch.empty(V, d_in, dtype=torch.float32, device=dev) if want_G_W else None
+    need = lib().dust_head_step_workspace(T, d_in, V, dt, int(Z is not None), int(want_G_W))
+    ws = workspace(need, dev)
+    _check(lib().dust_head_step(_opt(X, "X"), _opt(W, "W"), dt, _opt(Z, "Z", torch.float32),
+                                _dev(targets, "targets", torch.int32), T, d_in, V, Vc, noise.c(), _opt(c, "c"),
+                                _dev(g_hat, "g_hat", torch.float32), _opt(g16, "g_hat_bf16"), _opt(G_W, "G_W"),
+                                int(bool(accumulate)), ws.data_ptr(), ws.numel(), _stream()))
+    return {"g_hat": g_hat, "c": c, "g_hat_bf16": g16, "G_W": G_W}
+
+
+# ------------------------------------------------------------------ harness
+def noise_fill(noise: Noise, t0: int, n_tok: int, j0: int, n_ch: int, stream_id: int = 0, device="cuda"):
+    out = torch.empty(noise.draw_count, n_tok, n_ch, dtype=torch.float32, device=device)
+    _check(lib().dust_noise_fill(noise.c(), stream_id, t0, n_tok, j0, n_ch, out.data_ptr(), _stream()))
+    return out
+
+
+def synth_costs(u: torch.Tensor, noise: Noise, eps_scale: float = 0.01, out: torch.Tensor | None = None):
+    T, d_out = u.shape
+    c = torch.empty(noise.draw_count, T, dtype=torch.float32, device=u.device) if out is None else out
+    _check(lib().dust_synth_costs(_dev(u, "u", torch.float32), T, d_out, noise.c(), float(eps_scale),
+                                  _dev(c, "c", torch.float32), _stream()))
+    return c
+
+
+def toy_suffix_losses(Y, seq_offsets, Wq, Wk, Wv, Wo, Wout, targets, noise: Noise):
+    """Returns (loss [draw_count + 1][T] with row 0 clean, c [draw_count][T])."""
+    T, d = Y.shape
+    dh, V = Wq.shape[0], Wout.shape[0]
+    dev = Y.device
+    loss = torch.empty(noise.draw_count + 1, T, dtype=torch.float32, device=dev)
+    c = torch.empty(noise.draw_count, T, dtype=torch.float32, device=dev)
+    ws = workspace(lib().dust_toy_suffix_workspace(noise.draw_count, T, d, dh, V), dev)
+    f32 = torch.float32
+    _check(lib().dust_toy_suffix_losses(_dev(Y, "Y", f32), T, d, _dev(seq_offsets, "seq_offsets", torch.int32),
+                                        seq_offsets.numel() - 1, _dev(Wq, "Wq", f32), _dev(Wk, "Wk", f32),
+                                        _dev(Wv, "Wv", f32), _dev(Wo, "Wo", f32), dh, _dev(Wout, "Wout", f32), V,
+                                        _dev(targets, "targets", torch.int32), noise.c(), loss.data_ptr(),
+                                        c.data_ptr(), ws.data_ptr(), ws.numel(), _stream()))
+    return loss, c

@@ -1,0 +1,517 @@
+#!/usr/bin/env python
+"""Benchmark of the Dust estimator hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--draws K]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+for each hidden linear layer of the workload, the reward scan (a4), the
+noise-regenerating draw reduction (a1 + a5) and the weight estimate G_W (a6);
+for the LM head, the clean logits (a2, tcgen05), the fused perturbed cross
+entropy and its draw reduction over all vocabulary chunks (a1 + a3 + a5) and
+the head's G_W (a6).  The synthetic costs c that stand in for the perturbed
+forward of the hidden layers are produced once, before timing (harness).
+
+Metric: draws x tokens per second summed over the layers of one step,
+value = sum_layers K * T * N_ranks / max-over-ranks step time.  Every rank
+processes its own batch (weak scaling, data parallel); with N > 1 the weight
+estimates are summed over ranks by one NCCL all-reduce per step.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from activation_perturbation_es_b200 import inputs as I  # noqa: E402
+
+DEFAULT_WORKLOAD = I.SCALED.name
+METRIC = "Dust draws×tokens/s per layer step"
+UNIT = "draws×tokens/s"
+
+# Algorithmic work per element of the ALU-bound kernels, counted from the
+# operation sequence of the noise specification (one lane-operation per
+# primitive: integer mul-hi/lo, xor, shift, and/or, add, select; fp add, mul,
+# fma, div, sqrt; an exp-family function counts as one).
+#   Philox4x32-10: 10 rounds x (2 wide products = 4, 4 xors) = 80 per 4 Gaussians -> 20
+#   Box-Muller pair: uniforms 3, ln 18, rho 2, angle 8, sin/cos 12, octant
+#   swap 5, signs 8, products 2 = 58 per 2 Gaussians -> 29
+OPS_PER_GAUSSIAN = 49
+OPS_A5 = OPS_PER_GAUSSIAN + 1          # + the FMA into g
+OPS_HEAD = OPS_PER_GAUSSIAN + 4        # + sigma*a, expm1, FMA into S, FMA into g
+LANES_PER_SM = 128
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=3)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(I.WORKLOADS))
+    p.add_argument("--draws", type=int, default=0, help="override the workload's K")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "sm_max_mhz": d.get("sm_max_mhz", 1965.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0,
+            "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    import torch.distributed as dist
+    if world > 1:
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    import torch
+    import torch.distributed as dist
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ the step
+class Step:
+    """Device-resident buffers and the sequence of C-ABI calls of one step."""
+
+    def __init__(self, w: I.Workload, K: int, rank: int, world: int):
+        import torch
+        from activation_perturbation_es_b200 import dust
+        self.torch, self.dust, self.w, self.K, self.world = torch, dust, w, K, world
+        dev = torch.device("cuda", torch.cuda.current_device())
+        self.dev = dev
+        bf = torch.bfloat16
+        T = w.T
+        self.off = torch.from_numpy(I.uniform_offsets(w.n_seq, w.seq_len)).to(dev)
+        self.hidden = []
+        self.host = {}          # pinned host copies of every per-step input (for e2e)
+        for hl in w.hidden:
+            li = I.layer_inputs(w, hl, seed_offset=rank * 7919)
+            nz = dust.Noise(w.seed + rank, hl.layer, 0, K, K, w.sigma)
+            u = torch.from_numpy(li["u"]).to(dev)
+            c = dust.synth_costs(u, nz, w.eps_scale)          # harness: stands in for the perturbed forward
+            del u
+            X = torch.from_numpy(li["X"]).to(dev, bf)
+            L = {"hl": hl, "nz": nz, "c": c, "X": X,
+                 "r": torch.empty_like(c),
+                 "g": torch.empty(T, hl.d_out, dtype=torch.float32, device=dev),
+                 "g16": torch.empty(T, hl.d_out, dtype=bf, device=dev),
+                 "G": torch.empty(hl.d_out, hl.d_in, dtype=torch.float32, device=dev)}
+            self.hidden.append(L)
+        self.head = None
+        if w.V:
+            hi = I.head_inputs(w, seed_offset=rank * 7919)
+            nz = dust.Noise(w.seed + rank, w.head_layer, 0, K, K, w.sigma)
+            self.head = {"nz": nz, "X": torch.from_numpy(hi["X"]).to(dev, bf),
+                         "W": torch.from_numpy(hi["W"]).to(dev, bf),
+                         "y": torch.from_numpy(hi["y"]).to(dev),
+                         "Z": torch.empty(T, w.V, dtype=torch.float32, device=dev),
+                         "g": torch.empty(T, w.V, dtype=torch.float32, device=dev),
+                         "g16": torch.empty(T, w.V, dtype=bf, device=dev),
+                         "G": torch.empty(w.V, w.head_d, dtype=torch.float32, device=dev)}
+        torch.cuda.synchronize()
+        self.stage_names = []
+        for L in self.hidden:
+            n = L["hl"].name
+            self.stage_names += [f"{n}:scan", f"{n}:estimate", f"{n}:weight_grad"]
+        if self.head:
+            self.stage_names += ["head:logits", "head:ce_estimate", "head:weight_grad"]
+        self.events = None
+
+    def units(self):
+        return self.K * self.w.T * (len(self.hidden) + (1 if self.head else 0))
+
+    def make_events(self, n_steps):
+        ev = self.torch.cuda.Event
+        self.events = [[ev(enable_timing=True) for _ in range(len(self.stage_names) + 1)] for _ in range(n_steps)]
+
+    def run(self, step_idx=None):
+        dust = self.dust
+        evs = self.events[step_idx] if step_idx is not None else None
+        i = 0
+
+        def mark():
+            nonlocal i
+            if evs is not None:
+                evs[i].record()
+            i += 1
+
+        for L in self.hidden:
+            hl = L["hl"]
+            mark()
+            dust.reward_scan(L["c"], self.off, self.w.gamma, out=L["r"])
+            mark()
+            dust.layer_estimate(L["r"], True, self.off, self.w.gamma, L["nz"], hl.d_out, g_hat=L["g"],
+                                g_hat_bf16=L["g16"])
+            mark()
+            dust.weight_grad(L["g16"], L["X"], G_W=L["G"])
+        if self.head:
+            H = self.head
+            mark()
+            dust.logits(H["X"], H["W"], Z=H["Z"])
+            mark()
+            # row statistics + all chunk passes (a3 + a5) on the cached logits of a2
+            dust.head_step(H["y"], self.w.Vc, H["nz"], Z=H["Z"], g_hat=H["g"], g_hat_bf16=H["g16"])
+            mark()
+            dust.weight_grad(H["g16"], H["X"], G_W=H["G"])
+        mark()
+        if self.world > 1:
+            self.allreduce()
+
+    def allreduce(self):
+        import torch.distributed as dist
+        for L in self.hidden:
+            dist.all_reduce(L["G"])
+        if self.head:
+            dist.all_reduce(self.head["G"])
+
+    def stage_times(self, n_steps):
+        """Mean ms per stage over the timed steps."""
+        out = np.zeros(len(self.stage_names))
+        for s in range(n_steps):
+            e = self.events[s]
+            for k in range(len(self.stage_names)):
+                out[k] += e[k].elapsed_time(e[k + 1])
+        return out / n_steps
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return reference_arm(args)
+    import torch
+    world, rank, local = dist_setup(args)
+    w = I.WORKLOADS[args.workload]
+    K = args.draws or w.K
+    peaks = load_peaks()
+    step = Step(w, K, rank, world)
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    step.make_events(args.steps)
+    gpu_id = torch.cuda.get_device_properties(torch.cuda.current_device()).uuid
+    gpu_id = f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else str(gpu_id)
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for s in range(args.steps):
+            step.run(s)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms_total = max_over_ranks(t0.elapsed_time(t1), world)
+    ms_step = ms_total / args.steps
+    value = step.units() * world / (ms_step / 1e3)
+    stages = step.stage_times(args.steps)
+    clocks = clk.summary()
+
+    kernels = kernel_report(step, stages, peaks, clocks)
+    dominant = max(kernels, key=lambda k: k["ms"])
+    e2e = None if args.no_e2e else e2e_run(step, args, world)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, K, budget_s=20.0)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32 (noise, CE, reduction); bf16 in / f32 acc (tcgen05 GEMMs)",
+            "data": "synthetic (seeded; inputs > L2, no flush needed)",
+            "config": {"workload": w.name, "tokens_per_rank": w.T, "n_seq": w.n_seq, "seq_len": w.seq_len,
+                       "draws": K, "sigma": w.sigma, "gamma_hidden": w.gamma,
+                       "hidden": [[h.d_in, h.d_out] for h in w.hidden],
+                       "head": {"d": w.head_d, "V": w.V, "Vc": w.Vc} if w.V else None,
+                       "parallelism": f"dp{world}", "l2": "inputs larger than L2 (126 MB); no flush"},
+            "roofline": {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+            | {"kernel": dominant["name"], "clock_mhz_for_peak": dominant.get("clock_mhz_for_peak"),
+               "peak_source": dominant.get("peak_source")},
+            "kernels": kernels,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step(step) * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def launches_per_step(step):
+    """Kernels of this library launched per step (counted from the call sequence)."""
+    n = 0
+    for L in step.hidden:
+        n += 1                                   # reward scan
+        n += 1                                   # draw reduction
+        n += 1 if step.dust.lib().dust_weight_grad_workspace(step.w.T, L["hl"].d_in, L["hl"].d_out, 1) <= 256 else 2
+    if step.head:
+        n += 1                                   # logits GEMM
+        n += 2                                   # row stats + chunk passes
+        n += 1 if step.dust.lib().dust_weight_grad_workspace(step.w.T, step.w.head_d, step.w.V, 1) <= 256 else 2
+    return n
+
+
+def kernel_report(step, stages, peaks, clocks):
+    w, K, T = step.w, step.K, step.w.T
+    f_peak = peaks["sm_max_mhz"]
+    alu_peak = 148 * LANES_PER_SM * f_peak * 1e6 / 1e12          # Tops/s
+    out = []
+    names = step.stage_names
+    for name, ms in zip(names, stages):
+        layer, kind = name.split(":")
+        rec = {"name": name, "ms": float(ms)}
+        if layer == "head":
+            d_in, d_out = w.head_d, w.V
+        else:
+            hl = next(h for h in w.hidden if h.name == layer)
+            d_in, d_out = hl.d_in, hl.d_out
+        if kind == "scan":
+            byts = 8.0 * K * T
+            ach = byts / (ms / 1e3) / 1e9
+            rec |= {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": ach / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes": byts}
+        elif kind in ("weight_grad", "logits"):
+            fl = 2.0 * T * d_in * d_out
+            ach = fl / (ms / 1e3) / 1e12
+            rec |= {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": ach / peaks["bf16_tflops"], "traffic": None, "algorithmic_flops": fl}
+        else:
+            ops_el = OPS_HEAD if layer == "head" else OPS_A5
+            ops = float(K) * T * d_out * ops_el
+            ach = ops / (ms / 1e3) / 1e12
+            rec |= {"bound": "alu", "achieved": ach, "peak": alu_peak, "unit": "Tops/s",
+                    "frac": ach / alu_peak, "traffic": None, "algorithmic_ops": ops,
+                    "ops_per_element": ops_el, "clock_mhz_for_peak": f_peak,
+                    "gaussians_per_s": float(K) * T * d_out / (ms / 1e3),
+                    "peak_source": "148 SMs x 128 lanes x max SM clock (one lane-op per lane per clock)"}
+        out.append(rec)
+    return out
+
+
+# ------------------------------------------------------------------ end to end
+def e2e_run(step, args, world):
+    """Same metric through the public API with host buffers: every step copies its
+    inputs from pinned host memory and reads the weight estimates back."""
+    import torch
+    hosts = []
+    for L in step.hidden:
+        hosts.append((L["c"], L["c"].cpu().pin_memory()))
+        hosts.append((L["X"], L["X"].cpu().pin_memory()))
+    if step.head:
+        for k in ("X", "W", "y"):
+            hosts.append((step.head[k], step.head[k].cpu().pin_memory()))
+    outs = [L["G"] for L in step.hidden] + ([step.head["G"]] if step.head else [])
+    outs_h = [o.cpu().pin_memory() for o in outs]
+    h2d = sum(h.numel() * h.element_size() for _, h in hosts)
+    d2h = sum(o.numel() * o.element_size() for o in outs_h)
+
+    def one():
+        for dev_t, host_t in hosts:
+            dev_t.copy_(host_t, non_blocking=True)
+        step.run()
+        for o, oh in zip(outs, outs_h):
+            oh.copy_(o, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(1, min(args.steps, 3))
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(n):
+        one()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(t0.elapsed_time(t1), world) / n
+    return {"value": step.units() * world / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": n}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(w: I.Workload, K: int, n_tok: int):
+    """Times the CPU oracle on a bounded sample of one step: for every layer, the
+    error estimate of n_tok tokens over all K draws and all output channels (and,
+    for hidden layers, their rewards from c).  Returns (seconds, draws x tokens
+    processed, extrapolated seconds for the full step)."""
+    import oracle
+    rs = np.random.Generator(np.random.PCG64(0))
+    off = I.uniform_offsets(w.n_seq, w.seq_len)
+    toks = np.sort(rs.choice(w.T, n_tok, replace=False)).astype(np.int32)
+    t_sample, units, t_full = 0.0, 0, 0.0
+    for hl in w.hidden:
+        # costs for the sampled tokens' sequences only (the rest of c is never read)
+        c = np.zeros((K, w.T), np.float32)
+        c[:, toks] = I.normal((K, n_tok), w.sigma, seed=hl.layer)
+        t = time.perf_counter()
+        oracle.layer_estimate(c, False, hl.d_out, off, w.gamma, w.seed, hl.layer, 0, K, w.sigma, toks)
+        dt = time.perf_counter() - t
+        t_sample += dt
+        units += K * n_tok
+        t_full += dt * w.T / n_tok
+    if w.V:
+        Z = I.normal((n_tok, w.V), 1.0, seed=99)
+        y = I.targets(n_tok, w.V, seed=98)
+        t = time.perf_counter()
+        oracle.head_step(Z, y, toks, w.Vc, w.seed, w.head_layer, 0, K, K, w.sigma, want_c=False)
+        dt = time.perf_counter() - t
+        t_sample += dt
+        units += K * n_tok
+        t_full += dt * w.T / n_tok
+    return t_sample, units, t_full
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, K, budget_s=20.0):
+    cores = cpu_cores()
+    n_tok = max(2, min(512, 2 * cores))
+    t_s, units, t_full = oracle_sample(w, K, n_tok)
+    n_layers = len(w.hidden) + (1 if w.V else 0)
+    return {"value": n_layers * K * w.T / t_full, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n_tok} sampled tokens per layer x all {K} draws x all channels "
+                      f"({len(w.hidden)} hidden layers + head), {t_s:.1f} s, extrapolated linearly in tokens",
+            "sample_seconds": t_s}
+
+
+def reference_arm(args):
+    """The CPU oracle as the reference arm: each step is a bounded sample of the
+    workload timed on the host cores; other ranks exit without work."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = I.WORKLOADS[args.workload]
+    K = args.draws or w.K
+    cores = cpu_cores()
+    n_tok = max(1, min(64, cores // 2))
+    for _ in range(args.warmup):
+        oracle_sample(w, K, max(1, n_tok // 4))
+    t_s, t_full, units = 0.0, 0.0, 0
+    for _ in range(args.steps):
+        a, u, f = oracle_sample(w, K, n_tok)
+        t_s += a
+        units += u
+        t_full += f
+    n_layers = len(w.hidden) + (1 if w.V else 0)
+    value = n_layers * K * w.T * args.steps / t_full
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_full / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+            "data": "synthetic", "config": {"workload": w.name, "draws": K, "tokens_per_rank": w.T},
+            "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": cores,
+                             "sample": f"{n_tok} tokens per layer per step, all draws and channels, "
+                                       f"extrapolated linearly in tokens"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,203 @@
+/*
+ * dust.h -- C ABI of libdust.so, the B200 (sm_100a) hot path of the Dust
+ * virtual-population gradient estimator for one linear layer and for the LM
+ * head.
+ *
+ * Sources.  The method is stated in the cnblogs explainer "Dust: Pretraining
+ * Transformers Without Backpropagation" (cnblogs.com/32bin/p/23212811):
+ *   [CA]  section "信用分配：一次前向，两种奖励" (credit assignment):
+ *         noise a_t ~ N(0, I) added as y_t + sigma a_t; centred per-token
+ *         loss change c_s = l~_s - l_s; discounted reward
+ *         r_t = sum_{s>=t} gamma^(s-t) c_s (reward equation); output-side
+ *         error g_t = -(1/(K sigma)) sum_i r_t^(i) a_t^(i) (error equation);
+ *         weight estimate G_W = sum_t g_t x_t^T (weight equation).
+ *   [IS3] section "真正的工作量：压住干扰" (interference suppression), third
+ *         measure: the LM head perturbs the cached logits and recomputes only
+ *         the cross entropy over one chunk of the vocabulary.
+ * The noise a is regenerated from its coordinates by Philox4x32-10 (Salmon et
+ * al., SC'11) and a Box-Muller transform with series ln/sin/cos; the exact
+ * operation sequence is the library's noise specification and is identical,
+ * bit for bit, to the one any conforming implementation produces.
+ *
+ * Conventions (every entry point):
+ *   - All tensors are row-major, last index contiguous, in DEVICE memory of
+ *     the current CUDA device unless a parameter says "host".
+ *   - The caller owns every buffer, including the workspace.  The library
+ *     never allocates, frees or synchronises; every call only enqueues work
+ *     on `stream` (a cudaStream_t passed as void*; NULL = legacy default
+ *     stream) and returns.
+ *   - Device pointers must be 16-byte aligned (DUST_ERR_ALIGNMENT otherwise).
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid call launches nothing and returns a non-zero status.
+ *     dust_last_error() then gives a message (thread-local).
+ *   - Sequence offsets `seq_offsets` (device, int32 [n_seq + 1]) are read
+ *     only by the kernels: offsets[0] = 0, non-decreasing, offsets[n_seq] = T.
+ *     Kernels clamp every offset into [0, T], so offsets that break these
+ *     rules cannot make a kernel touch memory outside its tensors, but the
+ *     results are then unspecified; dust_check_offsets() validates a host
+ *     copy.
+ */
+#ifndef DUST_H
+#define DUST_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DUST_ABI_VERSION 1
+
+typedef enum {
+    DUST_OK = 0,
+    DUST_ERR_INVALID_ARG = 1,   /* a size, pointer or value is out of range */
+    DUST_ERR_UNSUPPORTED = 2,   /* a valid combination this build does not implement */
+    DUST_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned */
+    DUST_ERR_WORKSPACE = 4,     /* ws_bytes below the size the *_workspace query returns */
+    DUST_ERR_CUDA = 5,          /* a CUDA launch or driver call failed */
+    DUST_ERR_TIMEOUT = 6        /* a kernel's bounded wait ran out (reported by dust_poll_status) */
+} dust_status;
+
+typedef enum { DUST_F32 = 0, DUST_BF16 = 1 } dust_dtype;
+
+/* Which draws of which layer a call handles.  The noise element of draw i,
+ * token t, channel j is a(seed, layer, i, t, j); a call handles the global
+ * draws [draw_begin, draw_begin + draw_count) and scales by the whole
+ * population K_total, so that splitting the draws of one estimate over several
+ * calls (accumulate = 1) gives the same sum [CA, error equation]. */
+typedef struct {
+    uint32_t seed;        /* Philox key word 0 */
+    uint32_t layer;       /* Philox key word 1 (one value per perturbed layer) */
+    uint32_t draw_begin;  /* first global draw index handled by this call */
+    uint32_t draw_count;  /* number of draws handled by this call (> 0) */
+    uint32_t K_total;     /* population size K of the 1/(K sigma) scale (> 0) */
+    float sigma;          /* noise scale (> 0, finite) */
+} dust_noise;
+
+/* ------------------------------------------------------------------ status */
+
+const char *dust_status_string(dust_status s);
+/* Message of the last failed call on this host thread ("" if none). */
+const char *dust_last_error(void);
+int dust_abi_version(void);
+
+/* Host-side validation of sequence offsets (HOST pointer, n_seq + 1 entries). */
+dust_status dust_check_offsets(const int32_t *seq_offsets_host, int n_seq, int T);
+
+/* Reads and clears the device status word at the start of a workspace that a
+ * previous call on `stream` was given (synchronises `stream`).  Returns
+ * DUST_ERR_TIMEOUT if a kernel's bounded wait ran out, else DUST_OK. */
+dust_status dust_poll_status(void *ws, void *stream);
+
+/* ------------------------------------------------------------------ a4: reward
+ * [CA, reward equation] r[i][t] = sum_{s>=t, s in seq(t)} gamma^(s-t) c[i][s].
+ * c, r: [K][T] fp32; r may alias c (in place).  The sum stays inside the
+ * token's sequence (causal attention does not cross sequences).  gamma = 0
+ * gives r = c bit for bit.  0 <= gamma <= 1.  No workspace. */
+dust_status dust_reward_scan(const float *c, float *r, int K, int T,
+                             const int32_t *seq_offsets, int n_seq, float gamma,
+                             void *stream);
+
+/* ------------------------------------------------------------------ a5: error
+ * [CA, error equation] g_hat[t][j] (+)= -(1/(K_total sigma))
+ *     sum_{k < draw_count} r[k][t] a(seed, layer, draw_begin + k, t, j).
+ * c_or_r: [draw_count][T] fp32, row k belongs to draw draw_begin + k.  If
+ * is_r == 0 it holds the costs c and the reward scan (a4) runs first into the
+ * workspace (skipped when gamma == 0, where r = c); otherwise it holds r.
+ * g_hat: [T][d_out] fp32, overwritten (accumulate = 0) or added to
+ * (accumulate = 1).  g_hat_bf16: nullable [T][d_out] bf16, receives
+ * round-to-nearest-even of the final g_hat.  Workspace:
+ * dust_layer_estimate_workspace(). */
+dust_status dust_layer_estimate(const float *c_or_r, int is_r, int T, int d_out,
+                                const int32_t *seq_offsets, int n_seq, float gamma,
+                                dust_noise nz, float *g_hat, void *g_hat_bf16,
+                                int accumulate, void *ws, size_t ws_bytes, void *stream);
+size_t dust_layer_estimate_workspace(int draw_count, int T, int d_out, int is_r, float gamma);
+
+/* ------------------------------------------------------------------ a6: weight
+ * [CA, weight equation] G_W[o][i] (+)= sum_t g_hat[t][o] X[t][i].
+ * g_hat: [T][d_out], X: [T][d_in], both of dtype `dt` (DUST_BF16 runs on the
+ * tcgen05 tensor cores with fp32 accumulation in TMEM and needs d_in and d_out
+ * multiples of 16 and pointers 128-byte aligned; DUST_F32 runs on fp32 CUDA
+ * cores).  G_W: [d_out][d_in] fp32 (the layout of W).  Split over T with a
+ * fixed-order reduction: results do not depend on the launch.
+ * Workspace: dust_weight_grad_workspace(). */
+dust_status dust_weight_grad(const void *g_hat, const void *X, dust_dtype dt,
+                             int T, int d_in, int d_out, float *G_W, int accumulate,
+                             void *ws, size_t ws_bytes, void *stream);
+size_t dust_weight_grad_workspace(int T, int d_in, int d_out, dust_dtype dt);
+
+/* ------------------------------------------------------------------ a2: logits
+ * Clean head forward Z[t][v] = sum_k X[t][k] W[v][k] (no bias), fp32 out.
+ * X: [T][d_in], W: [V][d_in] of dtype dt (bf16: tcgen05; f32: CUDA cores).
+ * Workspace: dust_logits_workspace(). */
+dust_status dust_logits(const void *X, const void *W, dust_dtype dt, int T, int d_in,
+                        int V, float *Z, void *ws, size_t ws_bytes, void *stream);
+size_t dust_logits_workspace(int T, int d_in, int V, dust_dtype dt);
+
+/* Per-token clean statistics of cached logits: lse[t] = log sum_v exp Z[t][v],
+ * ell[t] = lse[t] - Z[t][targets[t]] (the clean loss l_t).  ell nullable.
+ * targets: [T] int32 in [0, V). */
+dust_status dust_head_row_stats(const float *Z, const int32_t *targets, int T, int V,
+                                float *lse, float *ell, void *stream);
+
+/* ------------------------------------------------------------------ a2+a3+a5+a6: head
+ * [IS3] LM-head step over all V/Vc vocabulary chunks.  For chunk
+ * [v0, v0 + Vc) and draw i, the logits of the chunk are perturbed,
+ * z~ = z + sigma a(i, t, v) for v in the chunk, and the change of the
+ * full-vocabulary cross entropy is [CA] c = CE(z~, y) - CE(z, y), computed as
+ * log1p(sum_{v in chunk} p_v expm1(sigma a_v)) - sigma a_y [y in chunk] with
+ * p = softmax(z) (an exact identity).  With gamma = 0 (head) r = c and
+ * g_hat[t][v] (+)= -(1/(K_total sigma)) sum_i c a(i, t, v) for v in the chunk.
+ * Noise channel = global vocab id v, so results do not depend on Vc.
+ *   X: [T][d_in], W: [V][d_in] of dtype dt; used when Z is NULL (Z is then
+ *      recomputed into the workspace, a2) and when G_W is requested.
+ *   Z: nullable cached logits [T][V] fp32.
+ *   targets: [T] int32 in [0, V).
+ *   Vc: chunk width; must divide V; supported: a multiple of 128, <= 1024.
+ *   c_out: nullable [V/Vc][draw_count][T] fp32, the costs of every pass.
+ *   g_hat: [T][V] fp32 (overwritten, or added to when accumulate = 1).
+ *   g_hat_bf16: nullable [T][V] bf16 copy of the final g_hat.
+ *   G_W: nullable [V][d_in] fp32, overwritten with g_hat^T X (a6) computed
+ *      from the final g_hat (requires X).
+ * Workspace: dust_head_step_workspace(). */
+dust_status dust_head_step(const void *X, const void *W, dust_dtype dt, const float *Z,
+                           const int32_t *targets, int T, int d_in, int V, int Vc,
+                           dust_noise nz, float *c_out, float *g_hat, void *g_hat_bf16,
+                           float *G_W, int accumulate, void *ws, size_t ws_bytes,
+                           void *stream);
+size_t dust_head_step_workspace(int T, int d_in, int V, dust_dtype dt, int has_Z, int want_G_W);
+
+/* ------------------------------------------------------------------ harness / debug
+ * Noise: out[k][t][j] = a(seed, layer, draw_begin + k, t0 + t, j0 + j) from
+ * Philox stream `stream_id` (0: activation noise, 1: synthetic observation
+ * noise).  out: [draw_count][n_tok][n_ch] fp32. */
+dust_status dust_noise_fill(dust_noise nz, uint32_t stream_id, int t0, int n_tok,
+                            int j0, int n_ch, float *out, void *stream);
+
+/* Synthetic linear costs standing in for a perturbed forward:
+ * c[k][s] = sigma <u[s], a(draw_begin+k, s, .)> + eps_scale * a_stream1(draw_begin+k, s, 0).
+ * u: [T][d_out] fp32, c: [draw_count][T] fp32. */
+dust_status dust_synth_costs(const float *u, int T, int d_out, dust_noise nz,
+                             float eps_scale, float *c, void *stream);
+
+/* Toy causal suffix scoring a perturbed hidden linear layer (fp32 CUDA cores):
+ * y~ = Y + sigma a(draw), h = y~ + Attn(y~) Wo^T (one causal softmax head of
+ * width dh per sequence; q, k, v = y~ Wq^T, y~ Wk^T, y~ Wv^T, scores scaled by
+ * 1/sqrt(dh)), z = h Wout^T, loss = logsumexp(z) - z[target].
+ * Y: [T][d] clean layer output; Wq, Wk, Wv: [dh][d]; Wo: [d][dh]; Wout: [V][d].
+ * loss: [draw_count + 1][T]; row 0 is the clean loss, row 1 + k draw
+ * draw_begin + k.  If c is non-NULL it receives c[k][t] = row(1+k) - row(0).
+ * Supported: d <= 1024, dh <= 128, d % 4 == 0.  Workspace: dust_toy_suffix_workspace(). */
+dust_status dust_toy_suffix_losses(const float *Y, int T, int d, const int32_t *seq_offsets,
+                                   int n_seq, const float *Wq, const float *Wk, const float *Wv,
+                                   const float *Wo, int dh, const float *Wout, int V,
+                                   const int32_t *targets, dust_noise nz, float *loss, float *c,
+                                   void *ws, size_t ws_bytes, void *stream);
+size_t dust_toy_suffix_workspace(int draw_count, int T, int d, int dh, int V);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DUST_H */
