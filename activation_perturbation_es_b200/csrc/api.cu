@@ -114,6 +114,12 @@ cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 }  // namespace
 
+namespace dust {
+// Lets entry points defined in other translation units report through
+// dust_last_error().
+dust_status record_error(dust_status s, const char* msg) { return fail(s, "%s", msg); }
+}  // namespace dust
+
 extern "C" {
 
 const char* dust_status_string(dust_status s) {

@@ -62,6 +62,9 @@ cudaError_t run_toy_suffix(const float* Y, int T, int d, const int32_t* offs, in
                            const int32_t* targets, const dust_noise& nz, float* loss, float* c, void* ws,
                            cudaStream_t st);
 
+// error reporting for entry points outside api.cu
+dust_status record_error(dust_status s, const char* msg);
+
 // fp32 -> bf16 (RNE) copy
 cudaError_t launch_to_bf16(const float* src, void* dst, size_t n, cudaStream_t stream);
 

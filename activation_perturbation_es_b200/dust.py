@@ -61,6 +61,7 @@ _SIGS = {
     "dust_reward_scan": ([_vp, _vp, _i, _i, _vp, _i, _f, _vp], _i),
     "dust_layer_estimate": ([_vp, _i, _i, _i, _vp, _i, _f, _Noise, _vp, _vp, _i, _vp, _sz, _vp], _i),
     "dust_layer_estimate_workspace": ([_i, _i, _i, _i, _f], _sz),
+    "dust_layer_estimate_noalloc": ([_vp, _i, _i, _vp, _i, _f, _Noise, _vp, _vp, _i, _vp], _i),
     "dust_weight_grad": ([_vp, _vp, _i, _i, _i, _i, _vp, _i, _vp, _sz, _vp], _i),
     "dust_weight_grad_workspace": ([_i, _i, _i, _i], _sz),
     "dust_logits": ([_vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp], _i),
@@ -180,6 +181,26 @@ def layer_estimate(c_or_r: torch.Tensor, is_r: bool, seq_offsets, gamma: float, 
                                      float(gamma), noise.c(), _dev(g_hat, "g_hat", torch.float32),
                                      _opt(g_hat_bf16, "g_hat_bf16", torch.bfloat16), int(bool(accumulate)),
                                      ws.data_ptr(), ws.numel(), _stream()))
+    return g_hat, g_hat_bf16
+
+
+def layer_estimate_noalloc(c: torch.Tensor, seq_offsets, gamma: float, noise: Noise, d_out: int,
+                           g_hat: torch.Tensor | None = None, g_hat_bf16: torch.Tensor | None = None,
+                           accumulate: bool = False):
+    """dust_layer_estimate_noalloc: the estimate from costs c with the library's
+    static scratch instead of a workspace (for callers that cannot allocate).
+    Returns (g_hat, g_hat_bf16 or None)."""
+    nd, T = c.shape
+    if nd != noise.draw_count:
+        raise ValueError("c must have draw_count rows")
+    if g_hat is None:
+        g_hat = torch.empty(T, d_out, dtype=torch.float32, device=c.device)
+    offs = None if seq_offsets is None else _dev(seq_offsets, "seq_offsets", torch.int32)
+    n_seq = 1 if seq_offsets is None else seq_offsets.numel() - 1
+    _check(lib().dust_layer_estimate_noalloc(_dev(c, "c", torch.float32), T, d_out, offs, n_seq, float(gamma),
+                                             noise.c(), _dev(g_hat, "g_hat", torch.float32),
+                                             _opt(g_hat_bf16, "g_hat_bf16", torch.bfloat16),
+                                             int(bool(accumulate)), _stream()))
     return g_hat, g_hat_bf16
 
 

@@ -115,6 +115,31 @@ dust_status dust_layer_estimate(const float *c_or_r, int is_r, int T, int d_out,
                                 int accumulate, void *ws, size_t ws_bytes, void *stream);
 size_t dust_layer_estimate_workspace(int draw_count, int T, int d_out, int is_r, float gamma);
 
+/* Allocation-free form of dust_layer_estimate with is_r = 0, for callers that
+ * cannot call cudaMalloc: for example a plugin inside a host framework that
+ * owns all device memory and hands it only the device pointers of its inputs
+ * and outputs, or a caller whose memory pool is fully reserved.  The pages
+ * have no counterpart: it is a deployment variant of the same computation
+ * (reward scan into scratch, then the draw reduction) whose scratch for r is a
+ * fixed 16 MiB device array inside the library image instead of a workspace.
+ *   c: [draw_count][T] fp32 costs; other arguments as dust_layer_estimate.
+ *   Limit: draw_count * T <= 4194304 when gamma > 0 (DUST_ERR_WORKSPACE
+ *   otherwise, nothing launched); split the draws over calls with
+ *   accumulate = 1 for more.  gamma = 0 uses no scratch.
+ *   The array costs 16 MiB on every GPU that loads the library, until exit.
+ *   It is shared by all calls: calls whose kernels may overlap on the GPU race
+ *   on it and must be serialised by the caller.  It keeps the last call's
+ *   contents; nothing needs to start at zero (the scan rewrites every r the
+ *   reduction reads).
+ *   Set-up: the first call on a device looks the array's device address up
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.  The call allocates nothing (no cudaMalloc,
+ *   cudaFree or allocating library routine). */
+dust_status dust_layer_estimate_noalloc(const float *c, int T, int d_out,
+                                        const int32_t *seq_offsets, int n_seq, float gamma,
+                                        dust_noise nz, float *g_hat, void *g_hat_bf16,
+                                        int accumulate, void *stream);
+
 /* ------------------------------------------------------------------ a6: weight
  * [CA, weight equation] G_W[o][i] (+)= sum_t g_hat[t][o] X[t][i].
  * g_hat: [T][d_out], X: [T][d_in], both of dtype `dt` (DUST_BF16 runs on the
