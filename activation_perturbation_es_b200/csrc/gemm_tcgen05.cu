@@ -1,12 +1,415 @@
-// gemm_tcgen05.cu -- placeholder until the tcgen05 kernel lands.
+// gemm_tcgen05.cu -- bf16 x bf16 -> fp32 GEMM on the 5th-generation tensor
+// cores (tcgen05.mma, accumulator in TMEM), operands staged by TMA.
+//
+// Serves a6, the weight estimate G_W = g^T X (cnblogs Dust explainer, credit-
+// assignment section, weight equation: the same outer product with the same
+// input as backprop), and a2, the clean head logits Z = X W^T.
+//   a6: C[d_out][d_in] = sum_t g[t][o] X[t][i]: both operands are MN-major
+//       (the reduction index t is the row index of both tensors);
+//   a2: C[T][V] = sum_k X[t][k] W[v][k]: both operands are K-major.
+//
+// Tile 128 x BN (BN in {64, 128, 256}), 64-deep k blocks in a 4-stage ring.
+// One CTA of 4 warps per output tile and k slice:
+//   warp 0, one lane: TMA producer (cp.async.bulk.tensor, 128-byte swizzle,
+//           no multicast), one mbarrier per stage with expected bytes;
+//   warp 1, one lane: MMA issuer, 4 x tcgen05.mma (M = 128, N = BN, K = 16)
+//           per stage, tcgen05.commit frees the stage; warp 1 also allocates
+//           and frees the TMEM accumulator (BN fp32 columns);
+//   warps 0-3: epilogue, tcgen05.ld of its 32 TMEM lanes (rows), fp32 stores.
+// Split over k writes fp32 partial tiles that a second kernel sums in a fixed
+// order (deterministic).  Every mbarrier wait is bounded: when a bound runs
+// out the kernel records the workspace status word, drains its own copies and
+// MMAs (bounded too), frees TMEM and returns.
+#include <cuda.h>
+
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace dust {
-bool gemm_tc_supported(int, int, int, bool, bool) { return false; }
-int gemm_tc_splits(int, int, int) { return 1; }
-cudaError_t launch_gemm_tc(const void*, bool, int, const void*, bool, int, int, int, int, float*, int, int, float*,
-                           int, uint32_t*, cudaStream_t) {
-    return cudaErrorNotSupported;
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;          // bf16 elements = 128 bytes = one swizzle row
+constexpr int kStages = 4;
+constexpr int kThreads = 128;
+constexpr uint32_t kWaitLimit = 1u << 22;   // polls of a single mbarrier (with back-off: seconds)
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Bounded wait: false when the limit ran out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    for (uint32_t it = 0; it < kWaitLimit; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (it > 64) __nanosleep(256);
+    }
+    return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// 32 TMEM columns of the warp's 32 lanes -> 32 registers per thread
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor (sm_100): start >> 4 in bits [0,14),
+// leading byte offset >> 4 in [16,30), stride byte offset >> 4 in [32,46),
+// version 1 in [46,48), base offset 0, swizzle mode in [61,64) (2 = 128 B).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= 1ull << 46;
+    d |= 2ull << 61;
+    return d;
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator (bits [4,6) = 1), A and
+// B bf16 (bits [7,10) = 1, [10,13) = 1), A/B major (bit 15/16: 1 = MN-major),
+// N >> 3 in [17,23), M >> 4 in [24,29).
+__host__ __device__ constexpr uint32_t instr_desc(int N, bool a_mn, bool b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn) << 15) |
+           (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(kBM >> 4) << 24);
+}
+
+template <int BN>
+struct Smem {
+    static constexpr int kABytes = kBM * kBK * 2;   // 16 KB
+    static constexpr int kBBytes = BN * kBK * 2;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+// A: K-major (rows m, 128-byte K rows) or MN-major (two 64-wide MN atoms of
+// 64 K rows each).  Same for B with BN rows / BN/64 atoms.
+template <int BN, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, int M, int N,
+               int K, int k_per_split, float* __restrict__ C, int ldc, int accumulate, float* __restrict__ partial,
+               uint32_t* __restrict__ status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    using S = Smem<BN>;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * S::kStageBytes);
+    uint64_t* empty = full + kStages;
+    uint64_t* done = empty + kStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM;
+    const int kb = blockIdx.z * k_per_split;
+    const int ke = min(K, kb + k_per_split);
+    const int nk = ke > kb ? (ke - kb + kBK - 1) / kBK : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(done, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, BN);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    bool ok = true;
+    if (warp == 0 && lane == 0 && nk > 0) {
+        // ---------------- TMA producer
+        int issued = 0;
+        for (int it = 0; it < nk && ok; ++it) {
+            const int s = it % kStages;
+            if (it >= kStages && !mbar_wait(&empty[s], ((it / kStages) - 1) & 1)) { ok = false; break; }
+            if (*abort_flag) { ok = false; break; }
+            uint8_t* sa = smem + s * S::kStageBytes;
+            uint8_t* sb = sa + S::kABytes;
+            mbar_arrive_expect_tx(&full[s], S::kStageBytes);
+            const int k0 = kb + it * kBK;
+            if (A_MN) {
+                tma_load_2d(sa, &map_a, &full[s], m0, k0);
+                tma_load_2d(sa + 64 * kBK * 2, &map_a, &full[s], m0 + 64, k0);
+            } else {
+                tma_load_2d(sa, &map_a, &full[s], k0, m0);
+            }
+            if (B_MN) {
+#pragma unroll
+                for (int h = 0; h < BN / 64; ++h) tma_load_2d(sb + h * 64 * kBK * 2, &map_b, &full[s], n0 + 64 * h, k0);
+            } else {
+                tma_load_2d(sb, &map_b, &full[s], k0, n0);
+            }
+            issued = it + 1;
+        }
+        if (!ok) {
+            atomicExch(status, kStatusTimeout);
+            *abort_flag = 1;
+        }
+        // drain: the last (up to kStages) loads must land before the CTA exits
+        for (int it = issued > kStages ? issued - kStages : 0; it < issued; ++it)
+            mbar_wait(&full[it % kStages], (it / kStages) & 1);
+    } else if (warp == 1 && lane == 0 && nk > 0) {
+        // ---------------- MMA issuer
+        constexpr uint32_t idesc = instr_desc(BN, A_MN, B_MN);
+        for (int it = 0; it < nk; ++it) {
+            const int s = it % kStages;
+            if (!mbar_wait(&full[s], (it / kStages) & 1) || *abort_flag) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + s * S::kStageBytes);
+            const uint32_t sb = sa + S::kABytes;
+#pragma unroll
+            for (int j = 0; j < kBK / 16; ++j) {
+                // K-major: the 16-element k step is 32 bytes along the swizzled row;
+                // MN-major: it is 16 rows of 128 bytes.
+                const uint64_t ad = A_MN ? smem_desc(sa + j * 16 * 128, 64 * kBK * 2, 1024)
+                                         : smem_desc(sa + j * 32, 16, 1024);
+                const uint64_t bd = B_MN ? smem_desc(sb + j * 16 * 128, 64 * kBK * 2, 1024)
+                                         : smem_desc(sb + j * 32, 16, 1024);
+                tc_mma(tmem, ad, bd, idesc, (it > 0 || j > 0) ? 1u : 0u);
+            }
+            tc_commit(&empty[s]);
+        }
+        if (!ok) {
+            atomicExch(status, kStatusTimeout);
+            *abort_flag = 1;
+        }
+        tc_commit(done);   // arrives once every MMA issued above has completed
+    }
+    __syncwarp();
+
+    // ---------------- epilogue: TMEM -> registers -> global
+    bool have = nk > 0;
+    if (have) {
+        if (!mbar_wait(done, 0)) {
+            if (lane == 0) atomicExch(status, kStatusTimeout);
+            have = false;
+        }
+    }
+    have = have && !*abort_flag;
+    have = __all_sync(0xffffffffu, have);   // tcgen05.ld is warp-collective
+    tc_fence_after();
+    const int row = m0 + warp * 32 + lane;
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+        float v[32];
+        if (have) {
+            tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(c0), v);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+        }
+        if (row >= M) continue;
+        const int col = n0 + c0;
+        if (partial != nullptr) {
+            float* dst = partial + (static_cast<size_t>(blockIdx.z) * M + row) * N + col;
+            if (col + 32 <= N && (N & 3) == 0) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+            } else {
+                for (int i = 0; i < 32 && col + i < N; ++i) dst[i] = v[i];
+            }
+        } else {
+            float* dst = C + static_cast<size_t>(row) * ldc + col;
+            if (col + 32 <= N && (ldc & 3) == 0) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                    float4 o = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                    if (accumulate) {
+                        const float4 p = *reinterpret_cast<float4*>(dst + i);
+                        o.x += p.x; o.y += p.y; o.z += p.z; o.w += p.w;
+                    }
+                    *reinterpret_cast<float4*>(dst + i) = o;
+                }
+            } else {
+                for (int i = 0; i < 32 && col + i < N; ++i) dst[i] = accumulate ? dst[i] + v[i] : v[i];
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, BN);
+}
+
+// ------------------------------------------------------------------ host side
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+    static EncodeTiled fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor [outer][inner] with row pitch `ld` elements, box {64, box_outer}, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int inner, int outer, int ld, int box_outer) {
+    EncodeTiled enc = encode_fn();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+    const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_outer)};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int pick_bn(int N) { return N >= 256 ? 256 : (N > 64 ? 128 : 64); }
+
+template <int BN, bool A_MN, bool B_MN>
+cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int K, int kps, int splits,
+                     float* C, int ldc, int accumulate, float* partial, uint32_t* status, cudaStream_t st) {
+    auto kern = gemm_tc_kernel<BN, A_MN, B_MN>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<BN>::kBytes);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    const dim3 grid(static_cast<unsigned>(ceil_div(N, BN)), static_cast<unsigned>(ceil_div(M, kBM)),
+                    static_cast<unsigned>(splits));
+    kern<<<grid, kThreads, Smem<BN>::kBytes, st>>>(ma, mb, M, N, K, kps, C, ldc, accumulate,
+                                                    splits > 1 ? partial : nullptr, status);
+    return cudaGetLastError();
+}
+
+template <bool A_MN, bool B_MN>
+cudaError_t launch_bn(int bn, const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int K, int kps, int splits,
+                      float* C, int ldc, int accumulate, float* partial, uint32_t* status, cudaStream_t st) {
+    switch (bn) {
+        case 256: return launch_t<256, A_MN, B_MN>(ma, mb, M, N, K, kps, splits, C, ldc, accumulate, partial, status, st);
+        case 128: return launch_t<128, A_MN, B_MN>(ma, mb, M, N, K, kps, splits, C, ldc, accumulate, partial, status, st);
+        default: return launch_t<64, A_MN, B_MN>(ma, mb, M, N, K, kps, splits, C, ldc, accumulate, partial, status, st);
+    }
+}
+
+}  // namespace
+
+bool gemm_tc_supported(int M, int N, int K, bool a_kmajor, bool b_kmajor) {
+    if (M <= 0 || N <= 0 || K <= 0) return false;
+    if (encode_fn() == nullptr) return false;
+    // TMA: global row pitch a multiple of 16 bytes -> contiguous extent a multiple of 8
+    const bool a_ok = a_kmajor ? (K % 8 == 0) : (M % 8 == 0);
+    const bool b_ok = b_kmajor ? (K % 8 == 0) : (N % 8 == 0);
+    return a_ok && b_ok;
+}
+
+int gemm_tc_splits(int M, int N, int K) {
+    const long long tiles = ceil_div(M, kBM) * ceil_div(N, pick_bn(N));
+    const long long kblocks = ceil_div(K, kBK);
+    // enough CTAs for several waves over the SMs, slices of at least 8 k blocks
+    long long s = 1;
+    while (tiles * s < 4LL * kNumSMs && kblocks / (s * 2) >= 8 && s < 32) s *= 2;
+    return static_cast<int>(s);
+}
+
+cudaError_t launch_gemm_tc(const void* A, bool a_kmajor, int lda, const void* B, bool b_kmajor, int ldb, int M, int N,
+                           int K, float* C, int ldc, int accumulate, float* partial, int splits, uint32_t* status,
+                           cudaStream_t stream) {
+    if (!gemm_tc_supported(M, N, K, a_kmajor, b_kmajor)) return cudaErrorNotSupported;
+    const int bn = pick_bn(N);
+    CUtensorMap ma, mb;
+    // A: K-major [M][K] -> box {64 k, 128 rows}; MN-major [K][M] -> box {64 m, 64 k rows}
+    const bool okA = a_kmajor ? make_map(&ma, A, K, M, lda, kBM) : make_map(&ma, A, M, K, lda, kBK);
+    const bool okB = b_kmajor ? make_map(&mb, B, K, N, ldb, bn) : make_map(&mb, B, N, K, ldb, kBK);
+    if (!okA || !okB) return cudaErrorInvalidValue;
+    const int kps = static_cast<int>(ceil_div(ceil_div(K, splits), kBK) * kBK);
+    cudaError_t e;
+    if (!a_kmajor && !b_kmajor)
+        e = launch_bn<true, true>(bn, ma, mb, M, N, K, kps, splits, C, ldc, accumulate, partial, status, stream);
+    else if (a_kmajor && b_kmajor)
+        e = launch_bn<false, false>(bn, ma, mb, M, N, K, kps, splits, C, ldc, accumulate, partial, status, stream);
+    else if (a_kmajor)
+        e = launch_bn<false, true>(bn, ma, mb, M, N, K, kps, splits, C, ldc, accumulate, partial, status, stream);
+    else
+        e = launch_bn<true, false>(bn, ma, mb, M, N, K, kps, splits, C, ldc, accumulate, partial, status, stream);
+    if (e != cudaSuccess || splits == 1) return e;
+    return launch_splitk_reduce(partial, splits, M, N, C, ldc, accumulate, stream);
+}
+
 }  // namespace dust

@@ -1,0 +1,52 @@
+"""Data-parallel plumbing for the estimator (host side, torch.distributed).
+
+The estimator shards two ways without changing what it computes:
+  * by sequences (data parallel): each rank owns whole sequences -- the reward
+    scan never crosses a sequence -- and the weight estimates of all ranks are
+    summed, G_W = sum_t g_t x_t^T over the global batch (cnblogs Dust
+    explainer, credit-assignment section, weight equation);
+  * by draws: each rank takes a contiguous range of the global draw indices
+    and scales by the whole population K_total, so the sum over ranks of the
+    partial estimates is the K-draw estimate (error equation, linear in the
+    draws).
+Either way the only exchange is one sum all-reduce per step.
+"""
+from __future__ import annotations
+
+import torch
+
+
+def draw_range(K: int, world: int, rank: int) -> tuple[int, int]:
+    """(draw_begin, draw_count) of `rank` when K draws are split over `world` ranks."""
+    if not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    b = K * rank // world
+    e = K * (rank + 1) // world
+    return b, e - b
+
+
+def sequence_range(n_seq: int, world: int, rank: int) -> tuple[int, int]:
+    """[first, last) sequence index of `rank` when n_seq whole sequences are split."""
+    if not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    return n_seq * rank // world, n_seq * (rank + 1) // world
+
+
+def allreduce_sum_(tensors, group=None) -> None:
+    """Sum each tensor over the ranks, in place, with one collective per dtype:
+    the tensors are packed into one flat buffer (fewer launches than one
+    all-reduce per layer)."""
+    import torch.distributed as dist
+    if not tensors or not dist.is_initialized() or dist.get_world_size(group) == 1:
+        return
+    by_dtype = {}
+    for t in tensors:
+        by_dtype.setdefault(t.dtype, []).append(t)
+    for ts in by_dtype.values():
+        flat = torch.cat([t.reshape(-1) for t in ts])
+        dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+        off = 0
+        for t in ts:
+            n = t.numel()
+            t.copy_(flat[off:off + n].view_as(t))
+            off += n

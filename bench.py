@@ -256,11 +256,8 @@ class Step:
             self.allreduce()
 
     def allreduce(self):
-        import torch.distributed as dist
-        for L in self.hidden:
-            dist.all_reduce(L["G"])
-        if self.head:
-            dist.all_reduce(self.head["G"])
+        from activation_perturbation_es_b200 import dp
+        dp.allreduce_sum_([L["G"] for L in self.hidden] + ([self.head["G"]] if self.head else []))
 
     def stage_times(self, n_steps):
         """Mean ms per stage over the timed steps."""

@@ -149,6 +149,28 @@ def test_weight_grad_bf16(orc, T, d_in, d_out):
     assert rel_err(G[rows], orc.weight_grad(g, X, rows=rows)) < 1e-4   # same bf16 inputs, fp32 accumulation
 
 
+@pytest.mark.parametrize("T,d_in,d_out", [(200, 24, 40), (777, 520, 136), (64, 64, 64)])
+def test_weight_grad_bf16_ragged_and_accumulate(orc, T, d_in, d_out):
+    """Tensor-core path with tails in every dimension (M, N not multiples of the
+    tile, T not a multiple of the 64-deep k block) and accumulate = 1."""
+    g = I.bf16_round(I.normal((T, d_out), 1.0, seed=T + 5))
+    X = I.bf16_round(I.normal((T, d_in), 1.0, seed=T + 6))
+    G0 = I.normal((d_out, d_in), 1.0, seed=T + 7)
+    G = cu(G0)
+    dust.weight_grad(cu(g, torch.bfloat16), cu(X, torch.bfloat16), G_W=G, accumulate=True)
+    ref = orc.weight_grad(g, X) + G0.astype(np.float64)
+    assert rel_err(host(G), ref) < 1e-5
+
+
+@pytest.mark.parametrize("T,d_in,V", [(1000, 64, 520), (256, 1024, 4096)])
+def test_logits_bf16_tensor_cores(orc, T, d_in, V):
+    X = I.bf16_round(I.normal((T, d_in), 1.0, seed=T))
+    W = I.bf16_round(I.normal((V, d_in), 1.0 / np.sqrt(d_in), seed=V))
+    Z = dust.logits(cu(X, torch.bfloat16), cu(W, torch.bfloat16))
+    toks = np.arange(0, T, 7)
+    assert rel_err(host(Z)[toks], orc.logits(X, W, toks)) < 1e-5
+
+
 @pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
 def test_logits_and_row_stats(orc, dt):
     T, d_in, V = 300, 64, 512
