@@ -161,6 +161,13 @@ dust_status dust_poll_status(void* ws, void* stream) {
     return fail(DUST_ERR_TIMEOUT, "a kernel's bounded wait ran out (status word 0x%08x)", word);
 }
 
+dust_status dust_selftest_bounded_wait(void* ws, uint32_t polls, void* stream) {
+    DUST_REQUIRE(ws != nullptr, DUST_ERR_INVALID_ARG, "ws must not be NULL");
+    DUST_REQUIRE(polls >= 1 && polls <= (1u << 20), DUST_ERR_INVALID_ARG, "polls must be in [1, 2^20]");
+    return cuda_status(dust::launch_bounded_wait_selftest(static_cast<uint32_t*>(ws), polls, as_stream(stream)),
+                       "dust_selftest_bounded_wait");
+}
+
 // ------------------------------------------------------------------ a4
 dust_status dust_reward_scan(const float* c, float* r, int K, int T, const int32_t* seq_offsets, int n_seq,
                              float gamma, void* stream) {
@@ -363,6 +370,16 @@ dust_status dust_noise_fill(dust_noise nz, uint32_t stream_id, int t0, int n_tok
     DUST_TRY(check_ptr(out, "out"));
     return cuda_status(dust::launch_noise_fill(nz, stream_id, t0, n_tok, j0, n_ch, out, as_stream(stream)),
                        "dust_noise_fill");
+}
+
+dust_status dust_box_muller_words(const uint32_t* a, const uint32_t* b, long long n, float* n_even, float* n_odd,
+                                  void* stream) {
+    DUST_REQUIRE(n > 0, DUST_ERR_INVALID_ARG, "n must be > 0");
+    DUST_TRY(check_ptr(a, "a"));
+    DUST_TRY(check_ptr(b, "b"));
+    DUST_TRY(check_ptr(n_even, "n_even"));
+    DUST_TRY(check_ptr(n_odd, "n_odd"));
+    return cuda_status(dust::launch_box_muller_words(a, b, n, n_even, n_odd, as_stream(stream)), "dust_box_muller_words");
 }
 
 dust_status dust_synth_costs(const float* u, int T, int d_out, dust_noise nz, float eps_scale, float* c, void* stream) {

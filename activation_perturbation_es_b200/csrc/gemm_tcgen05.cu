@@ -64,8 +64,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait: false when the limit ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    for (uint32_t it = 0; it < kWaitLimit; ++it) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = kWaitLimit) {
+    for (uint32_t it = 0; it < limit; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if (it > 64) __nanosleep(256);
     }
@@ -308,6 +308,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     if (warp == 1) tmem_dealloc(tmem, BN);
 }
 
+// One thread waits, with the pipeline's bounded-wait code, on an mbarrier that
+// nothing ever completes, so the wait runs out and the status word is set.
+__global__ void bounded_wait_selftest_kernel(uint32_t* status, uint32_t polls) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (!mbar_wait(&bar, 0, polls)) atomicExch(status, kStatusTimeout);
+    }
+}
+
 // ------------------------------------------------------------------ host side
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -369,6 +380,11 @@ cudaError_t launch_bn(int bn, const CUtensorMap& ma, const CUtensorMap& mb, int 
 }
 
 }  // namespace
+
+cudaError_t launch_bounded_wait_selftest(uint32_t* status, uint32_t polls, cudaStream_t stream) {
+    bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(status, polls);
+    return cudaGetLastError();
+}
 
 bool gemm_tc_supported(int M, int N, int K, bool a_kmajor, bool b_kmajor) {
     if (M <= 0 || N <= 0 || K <= 0) return false;

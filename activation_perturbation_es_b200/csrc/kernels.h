@@ -22,6 +22,8 @@ cudaError_t launch_layer_estimate(const float* r, int T, int d_out, const dust_n
 // a1 harness (noise_fill.cu)
 cudaError_t launch_noise_fill(const dust_noise& nz, uint32_t stream_id, int t0, int n_tok, int j0,
                               int n_ch, float* out, cudaStream_t stream);
+cudaError_t launch_box_muller_words(const uint32_t* a, const uint32_t* b, long long n, float* ne, float* no,
+                                    cudaStream_t stream);
 cudaError_t launch_synth_costs(const float* u, int T, int d_out, const dust_noise& nz,
                                float eps_scale, float* c, cudaStream_t stream);
 
@@ -46,6 +48,7 @@ cudaError_t launch_gemm_tc(const void* A, bool a_kmajor, int lda, const void* B,
                            int ldb, int M, int N, int K, float* C, int ldc, int accumulate,
                            float* partial, int splits, uint32_t* status, cudaStream_t stream);
 int gemm_tc_splits(int M, int N, int K);
+cudaError_t launch_bounded_wait_selftest(uint32_t* status, uint32_t polls, cudaStream_t stream);
 bool gemm_tc_supported(int M, int N, int K, bool a_kmajor, bool b_kmajor);
 
 // a2 row statistics + a3/a5 fused head (head.cu)

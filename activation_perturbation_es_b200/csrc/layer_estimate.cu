@@ -24,11 +24,18 @@ namespace dust {
 
 namespace {
 
-__device__ __forceinline__ void fma4(float4& acc, float r, const float4& a) {
-    acc.x = __fmaf_rn(r, a.x, acc.x);
-    acc.y = __fmaf_rn(r, a.y, acc.y);
-    acc.z = __fmaf_rn(r, a.z, acc.z);
-    acc.w = __fmaf_rn(r, a.w, acc.w);
+// acc += r * a for the 4 channels of one Philox call; r is folded into the
+// Box-Muller radius (r * rho once per pair instead of rho * cos and rho * sin).
+__device__ __forceinline__ void accumulate_quad(float4& acc, float r, uint32_t seed, uint32_t layer, uint32_t draw,
+                                                uint32_t token, uint32_t quad) {
+    const uint4 x = philox4x32_10(make_uint4(quad, token, draw, 0u), seed, layer);
+    const Polar p01 = box_muller_polar(x.x, x.y);
+    const Polar p23 = box_muller_polar(x.z, x.w);
+    const float r01 = r * p01.rho, r23 = r * p23.rho;
+    acc.x = __fmaf_rn(r01, p01.cos_t, acc.x);
+    acc.y = __fmaf_rn(r01, p01.sin_t, acc.y);
+    acc.z = __fmaf_rn(r23, p23.cos_t, acc.z);
+    acc.w = __fmaf_rn(r23, p23.sin_t, acc.w);
 }
 
 __global__ void __launch_bounds__(256)
@@ -46,14 +53,12 @@ layer_estimate_kernel(const float* __restrict__ r, int T, int d_out, int nq, uin
         for (; k + 2 <= nd; k += 2) {
             const float r0 = __ldg(rt + static_cast<size_t>(k) * T);
             const float r1 = __ldg(rt + static_cast<size_t>(k + 1) * T);
-            const float4 a0 = gauss4(seed, layer, draw_begin + k, t, q, 0);
-            const float4 a1 = gauss4(seed, layer, draw_begin + k + 1, t, q, 0);
-            fma4(acc0, r0, a0);
-            fma4(acc1, r1, a1);
+            accumulate_quad(acc0, r0, seed, layer, draw_begin + k, t, q);
+            accumulate_quad(acc1, r1, seed, layer, draw_begin + k + 1, t, q);
         }
         if (k < nd) {
             const float r0 = __ldg(rt + static_cast<size_t>(k) * T);
-            fma4(acc0, r0, gauss4(seed, layer, draw_begin + k, t, q, 0));
+            accumulate_quad(acc0, r0, seed, layer, draw_begin + k, t, q);
         }
         float4 out = make_float4((acc0.x + acc1.x) * scale, (acc0.y + acc1.y) * scale,
                                  (acc0.z + acc1.z) * scale, (acc0.w + acc1.w) * scale);

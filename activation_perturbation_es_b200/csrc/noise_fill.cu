@@ -30,6 +30,16 @@ __global__ void noise_fill_kernel(uint32_t seed, uint32_t layer, uint32_t stream
     }
 }
 
+__global__ void box_muller_words_kernel(const uint32_t* __restrict__ a, const uint32_t* __restrict__ b, long long n,
+                                        float* __restrict__ ne, float* __restrict__ no) {
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const float2 v = box_muller(a[i], b[i]);
+        ne[i] = v.x;
+        no[i] = v.y;
+    }
+}
+
 // Block: 8 warps; warp w owns token s = blockIdx.x * 8 + w, lane l owns draw
 // k = blockIdx.y * 32 + l, so the u row is a warp-wide broadcast.  The 8 x 32
 // results are transposed through shared memory into 32-byte runs of c.
@@ -83,6 +93,15 @@ cudaError_t launch_noise_fill(const dust_noise& nz, uint32_t stream_id, int t0, 
     noise_fill_kernel<<<static_cast<unsigned>(blocks < 65536 ? blocks : 65536), 256, 0, stream>>>(
         nz.seed, nz.layer, stream_id, nz.draw_begin, static_cast<int>(nz.draw_count), t0, n_tok, j0,
         n_ch, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_box_muller_words(const uint32_t* a, const uint32_t* b, long long n, float* ne, float* no,
+                                    cudaStream_t stream) {
+    if (n == 0) return cudaSuccess;
+    const long long blocks = ceil_div(n, 256);
+    box_muller_words_kernel<<<static_cast<unsigned>(blocks < 8 * 1184 ? blocks : 8 * 1184), 256, 0, stream>>>(a, b, n,
+                                                                                                            ne, no);
     return cudaGetLastError();
 }
 

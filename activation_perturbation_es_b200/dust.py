@@ -58,6 +58,7 @@ _SIGS = {
     "dust_abi_version": ([], _i),
     "dust_check_offsets": ([_vp, _i, _i], _i),
     "dust_poll_status": ([_vp, _vp], _i),
+    "dust_selftest_bounded_wait": ([_vp, _u, _vp], _i),
     "dust_reward_scan": ([_vp, _vp, _i, _i, _vp, _i, _f, _vp], _i),
     "dust_layer_estimate": ([_vp, _i, _i, _i, _vp, _i, _f, _Noise, _vp, _vp, _i, _vp, _sz, _vp], _i),
     "dust_layer_estimate_workspace": ([_i, _i, _i, _i, _f], _sz),
@@ -70,6 +71,7 @@ _SIGS = {
     "dust_head_step": ([_vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _Noise, _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp], _i),
     "dust_head_step_workspace": ([_i, _i, _i, _i, _i, _i], _sz),
     "dust_noise_fill": ([_Noise, _u, _i, _i, _i, _i, _vp, _vp], _i),
+    "dust_box_muller_words": ([_vp, _vp, C.c_longlong, _vp, _vp, _vp], _i),
     "dust_synth_costs": ([_vp, _i, _i, _Noise, _f, _vp, _vp], _i),
     "dust_toy_suffix_losses": ([_vp, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp, _Noise, _vp, _vp,
                                 _vp, _sz, _vp], _i),
@@ -146,6 +148,10 @@ def check_offsets(seq_offsets, T: int) -> None:
 
 def poll_status(ws: torch.Tensor) -> None:
     _check(lib().dust_poll_status(_dev(ws, "ws"), _stream()))
+
+
+def selftest_bounded_wait(ws: torch.Tensor, polls: int = 4096) -> None:
+    _check(lib().dust_selftest_bounded_wait(_dev(ws, "ws"), polls, _stream()))
 
 
 # ------------------------------------------------------------------ a4
@@ -283,6 +289,16 @@ def noise_fill(noise: Noise, t0: int, n_tok: int, j0: int, n_ch: int, stream_id:
     out = torch.empty(noise.draw_count, n_tok, n_ch, dtype=torch.float32, device=device)
     _check(lib().dust_noise_fill(noise.c(), stream_id, t0, n_tok, j0, n_ch, out.data_ptr(), _stream()))
     return out
+
+
+def box_muller_words(a: torch.Tensor, b: torch.Tensor):
+    """Box-Muller step of the noise generator on given word pairs (uint32 held in int32 tensors)."""
+    n = a.numel()
+    ne = torch.empty(n, dtype=torch.float32, device=a.device)
+    no = torch.empty(n, dtype=torch.float32, device=a.device)
+    _check(lib().dust_box_muller_words(_dev(a, "a", torch.int32), _dev(b, "b", torch.int32), n, ne.data_ptr(),
+                                       no.data_ptr(), _stream()))
+    return ne, no
 
 
 def synth_costs(u: torch.Tensor, noise: Noise, eps_scale: float = 0.01, out: torch.Tensor | None = None):

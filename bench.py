@@ -348,12 +348,34 @@ def launches_per_step(step):
     return n
 
 
+def load_traffic():
+    """ncu DRAM bytes per output unit from profiles/traffic.txt, for kernels whose
+    source is unchanged since the capture (sha1 prefix match); else absent."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    out = {}
+    if not os.path.exists(path):
+        return out
+    for ln in open(path):
+        if ln.startswith("#") or not ln.strip():
+            continue
+        kernel, per_unit, unit, src, sha = ln.split()
+        try:
+            cur = hashlib.sha1(open(os.path.join(ROOT, src), "rb").read()).hexdigest()[:len(sha)]
+        except OSError:
+            continue
+        if cur == sha:
+            out[kernel] = (float(per_unit), unit)
+    return out
+
+
 def kernel_report(step, stages, peaks, clocks):
     w, K, T = step.w, step.K, step.w.T
     f_peak = peaks["sm_max_mhz"]
     alu_peak = 148 * LANES_PER_SM * f_peak * 1e6 / 1e12          # Tops/s
     out = []
     names = step.stage_names
+    traffic = load_traffic()
     for name, ms in zip(names, stages):
         layer, kind = name.split(":")
         rec = {"name": name, "ms": float(ms)}
@@ -376,8 +398,13 @@ def kernel_report(step, stages, peaks, clocks):
             ops_el = OPS_HEAD if layer == "head" else OPS_A5
             ops = float(K) * T * d_out * ops_el
             ach = ops / (ms / 1e3) / 1e12
+            tkey = "head_chunk_kernel" if layer == "head" else "layer_estimate"
+            tr = traffic.get(tkey)
             rec |= {"bound": "alu", "achieved": ach, "peak": alu_peak, "unit": "Tops/s",
-                    "frac": ach / alu_peak, "traffic": None, "algorithmic_ops": ops,
+                    "frac": ach / alu_peak, "traffic": tr[0] * T * d_out if tr else None,
+                    "traffic_source": "profiles/traffic.txt (ncu small case, scaled by tokens x channels)"
+                    if tr else None,
+                    "algorithmic_ops": ops,
                     "ops_per_element": ops_el, "clock_mhz_for_peak": f_peak,
                     "gaussians_per_s": float(K) * T * d_out / (ms / 1e3),
                     "peak_source": "148 SMs x 128 lanes x max SM clock (one lane-op per lane per clock)"}

@@ -90,6 +90,14 @@ dust_status dust_check_offsets(const int32_t *seq_offsets_host, int n_seq, int T
  * DUST_ERR_TIMEOUT if a kernel's bounded wait ran out, else DUST_OK. */
 dust_status dust_poll_status(void *ws, void *stream);
 
+/* Failure-detection self-test: one thread waits, through the same bounded
+ * mbarrier wait the tcgen05 pipeline uses, on a barrier that nothing
+ * completes; after `polls` polls (1 .. 2^20, with back-off: well under a
+ * second) it gives up and sets the status word of `ws`, so that a following
+ * dust_poll_status(ws) returns DUST_ERR_TIMEOUT.  Nothing faults or hangs and
+ * the context stays usable. */
+dust_status dust_selftest_bounded_wait(void *ws, uint32_t polls, void *stream);
+
 /* ------------------------------------------------------------------ a4: reward
  * [CA, reward equation] r[i][t] = sum_{s>=t, s in seq(t)} gamma^(s-t) c[i][s].
  * c, r: [K][T] fp32; r may alias c (in place).  The sum stays inside the
@@ -200,6 +208,12 @@ size_t dust_head_step_workspace(int T, int d_in, int V, dust_dtype dt, int has_Z
  * noise).  out: [draw_count][n_tok][n_ch] fp32. */
 dust_status dust_noise_fill(dust_noise nz, uint32_t stream_id, int t0, int n_tok,
                             int j0, int n_ch, float *out, void *stream);
+
+/* The noise generator's Box-Muller step on caller-given Philox word pairs:
+ * (n_even[i], n_odd[i]) = transform(a[i], b[i]).  a, b: [n] uint32; outputs
+ * [n] fp32.  For exhaustive bit-exactness checks of the specification. */
+dust_status dust_box_muller_words(const uint32_t *a, const uint32_t *b, long long n,
+                                  float *n_even, float *n_odd, void *stream);
 
 /* Synthetic linear costs standing in for a perturbed forward:
  * c[k][s] = sigma <u[s], a(draw_begin+k, s, .)> + eps_scale * a_stream1(draw_begin+k, s, 0).
