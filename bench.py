@@ -515,9 +515,9 @@ def reference_arm(args):
     w = I.WORKLOADS[args.workload]
     K = args.draws or w.K
     cores = cpu_cores()
-    n_tok = max(1, min(64, cores // 2))
+    n_tok = max(1, min(128, cores))          # one sampled token per host thread and layer
     for _ in range(args.warmup):
-        oracle_sample(w, K, max(1, n_tok // 4))
+        oracle_sample(w, K, max(1, cores // 4))
     t_s, t_full, units = 0.0, 0.0, 0
     for _ in range(args.steps):
         a, u, f = oracle_sample(w, K, n_tok)
