@@ -63,20 +63,27 @@ row_stats_kernel(const float* __restrict__ Z, const int32_t* __restrict__ target
     }
 }
 
-// expm1(x) for |x| <= 0.125 by its Taylor series to x^5 (relative truncation
-// error below x^5/720 < 5e-8 there); the kernel uses it only when sigma is
-// small enough that |sigma a| stays in that range for every a the generator
-// can produce (|a| <= sqrt(46 ln 2) < 5.66).
-__device__ __forceinline__ float expm1_small(float x) {
-    float t = fmaf(x, 1.0f / 120.0f, 1.0f / 24.0f);
-    t = fmaf(x, t, 1.0f / 6.0f);
+// expm1(x) by its Taylor series, for the small |x| = |sigma a| of the head's
+// perturbations (|a| <= sqrt(46 ln 2) < 5.66 for every a the generator makes):
+//   tier 1, sigma <= 0.02  (|x| <= 0.114): to x^5, relative truncation < x^5/720 < 3e-8;
+//   tier 2, sigma <= 0.01  (|x| <= 0.057): to x^4, relative truncation < x^4/120 < 9e-8 < 2^-23.
+// Larger sigma (tier 0) uses expm1f.
+template <int TIER>
+__device__ __forceinline__ float expm1_series(float x) {
+    float t;
+    if (TIER == 1) {
+        t = fmaf(x, 1.0f / 120.0f, 1.0f / 24.0f);
+        t = fmaf(x, t, 1.0f / 6.0f);
+    } else {
+        t = fmaf(x, 1.0f / 24.0f, 1.0f / 6.0f);
+    }
     t = fmaf(x, t, 0.5f);
     return fmaf(x * x, t, x);
 }
 
 constexpr int kHeadWarps = 4;   // tokens per block
 
-template <int QPL, bool SMALL_SIGMA>   // channel quads per lane: Vc = 128 * QPL
+template <int QPL, int TIER>   // channel quads per lane: Vc = 128 * QPL; expm1 tier (see expm1_series)
 __global__ void __launch_bounds__(32 * kHeadWarps)
 head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
                   const int32_t* __restrict__ targets, int T, int V, int Vc, uint32_t seed, uint32_t layer,
@@ -124,7 +131,7 @@ head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
                 const float x = sigma * a[k][w];
-                S = fmaf(pv[w], SMALL_SIGMA ? expm1_small(x) : expm1f(x), S);
+                S = fmaf(pv[w], TIER == 0 ? expm1f(x) : expm1_series<TIER>(x), S);
             }
             if (i_own && k == ky) ay = wy == 0 ? n.x : (wy == 1 ? n.y : (wy == 2 ? n.z : n.w));
         }
@@ -171,22 +178,20 @@ cudaError_t launch_head_chunks(const float* Z, const float* lse, const int32_t* 
                                const dust_noise& nz, float* c_out, float* g, void* g_bf16, int accumulate,
                                cudaStream_t stream) {
     const dim3 grid(static_cast<unsigned>(ceil_div(T, kHeadWarps)), static_cast<unsigned>(V / Vc));
-    // |a| < 5.66 for every draw the generator produces: sigma <= 0.02 keeps
-    // |sigma a| within the series' range
-    const bool small_sigma = nz.sigma <= 0.02f;
+    // |a| < 5.66 for every draw the generator produces (see expm1_series)
+    const int tier = nz.sigma <= 0.01f ? 2 : (nz.sigma <= 0.02f ? 1 : 0);
     const float scale = static_cast<float>(-1.0 / (static_cast<double>(nz.K_total) * nz.sigma));
     auto* g16 = static_cast<__nv_bfloat16*>(g_bf16);
     const int nd = static_cast<int>(nz.draw_count);
-#define DUST_HEAD_LAUNCH(Q)                                                                                 \
-    do {                                                                                                    \
-        if (small_sigma)                                                                                    \
-            head_chunk_kernel<Q, true><<<grid, 32 * kHeadWarps, 0, stream>>>(                               \
-                Z, lse, targets, T, V, Vc, nz.seed, nz.layer, nz.draw_begin, nd, nz.sigma, scale, c_out, g, \
-                g16, accumulate);                                                                           \
-        else                                                                                                \
-            head_chunk_kernel<Q, false><<<grid, 32 * kHeadWarps, 0, stream>>>(                              \
-                Z, lse, targets, T, V, Vc, nz.seed, nz.layer, nz.draw_begin, nd, nz.sigma, scale, c_out, g, \
-                g16, accumulate);                                                                           \
+#define DUST_HEAD_TIER(Q, TIER_)                                                                           \
+    head_chunk_kernel<Q, TIER_><<<grid, 32 * kHeadWarps, 0, stream>>>(Z, lse, targets, T, V, Vc, nz.seed,     \
+                                                                      nz.layer, nz.draw_begin, nd, nz.sigma,  \
+                                                                      scale, c_out, g, g16, accumulate)
+#define DUST_HEAD_LAUNCH(Q)                          \
+    do {                                             \
+        if (tier == 2) DUST_HEAD_TIER(Q, 2);         \
+        else if (tier == 1) DUST_HEAD_TIER(Q, 1);    \
+        else DUST_HEAD_TIER(Q, 0);                   \
     } while (0)
     if (Vc % 128 != 0) return cudaErrorNotSupported;
     switch (Vc / 128) {
@@ -201,6 +206,7 @@ cudaError_t launch_head_chunks(const float* Z, const float* lse, const int32_t* 
         default: return cudaErrorNotSupported;
     }
 #undef DUST_HEAD_LAUNCH
+#undef DUST_HEAD_TIER
     return cudaGetLastError();
 }
 

@@ -215,17 +215,18 @@ def test_head_step_small_fp32(orc):
     assert rel_err(host(cached["G_W"]), G_ref) < FP32_TOL
 
 
-def test_head_step_chunks_and_split(orc):
+@pytest.mark.parametrize("sigma", [0.005, 0.02, 0.05])   # the three expm1 tiers of the head kernel
+def test_head_step_chunks_and_split(orc, sigma):
     """Several chunks, draw split with accumulate, target ids on chunk edges."""
     T, V, Vc, K = 40, 768, 256, 10
     Z = I.normal((T, V), 1.5, seed=5)
     y = I.targets(T, V, seed=6)
     y[:6] = [0, 255, 256, 511, 512, 767]
     gz, gy = cu(Z), cu(y)
-    full = dust.head_step(gy, Vc, dust.Noise(1, 2, 0, K, K, 0.02), Z=gz, want_c=True)
-    _head_check(orc, Z, y, np.arange(T), Vc, dust.Noise(1, 2, 0, K, K, 0.02), full, 1e-4)
-    part = dust.head_step(gy, Vc, dust.Noise(1, 2, 0, 4, K, 0.02), Z=gz)
-    dust.head_step(gy, Vc, dust.Noise(1, 2, 4, K - 4, K, 0.02), Z=gz, g_hat=part["g_hat"], accumulate=True)
+    full = dust.head_step(gy, Vc, dust.Noise(1, 2, 0, K, K, sigma), Z=gz, want_c=True)
+    _head_check(orc, Z, y, np.arange(T), Vc, dust.Noise(1, 2, 0, K, K, sigma), full, 1e-4)
+    part = dust.head_step(gy, Vc, dust.Noise(1, 2, 0, 4, K, sigma), Z=gz)
+    dust.head_step(gy, Vc, dust.Noise(1, 2, 4, K - 4, K, sigma), Z=gz, g_hat=part["g_hat"], accumulate=True)
     assert rel_err(host(part["g_hat"]), host(full["g_hat"])) < 1e-6
 
 
