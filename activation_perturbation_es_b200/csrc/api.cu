@@ -362,6 +362,67 @@ dust_status dust_head_step(const void* X, const void* W, dust_dtype dt, const fl
                     reinterpret_cast<float*>(region(ws, h.wpart)), status, st);
 }
 
+// ------------------------------------------------------------------ cosine tuner
+namespace {
+struct BpLayout {
+    size_t lse = 0, d = 0, part = 0, total = 0;
+    GemmPlan plan;
+};
+
+BpLayout bp_layout(int T, int d_in, int V, dust_dtype dt) {
+    BpLayout b;
+    Layout L;
+    b.plan = weight_grad_plan(T, d_in, V, dt);
+    b.lse = L.add(sizeof(float) * static_cast<size_t>(T));
+    b.d = L.add((dt == DUST_BF16 ? 2 : 4) * static_cast<size_t>(T) * V);
+    b.part = L.add(b.plan.partial_bytes);
+    b.total = L.off;
+    return b;
+}
+}  // namespace
+
+size_t dust_head_bp_grad_workspace(int T, int d_in, int V, dust_dtype dt) {
+    if (T <= 0 || d_in <= 0 || V <= 0) return dust::kStatusBytes;
+    return bp_layout(T, d_in, V, dt).total;
+}
+
+dust_status dust_head_bp_grad(const float* Z, const int32_t* targets, const void* X, dust_dtype dt, int T, int d_in,
+                              int V, float* G_bp, void* ws, size_t ws_bytes, void* stream) {
+    DUST_REQUIRE(dt == DUST_F32 || dt == DUST_BF16, DUST_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
+    DUST_REQUIRE(T > 0 && d_in > 0 && V > 0, DUST_ERR_INVALID_ARG, "T, d_in, V must be > 0");
+    DUST_TRY(check_ptr(Z, "Z"));
+    DUST_TRY(check_ptr(targets, "targets"));
+    DUST_TRY(check_ptr(X, "X"));
+    DUST_TRY(check_ptr(G_bp, "G_bp"));
+    DUST_TRY(check_ptr(ws, "ws"));
+    const BpLayout b = bp_layout(T, d_in, V, dt);
+    DUST_REQUIRE(ws_bytes >= b.total, DUST_ERR_WORKSPACE, "workspace %zu bytes < %zu", ws_bytes, b.total);
+    cudaStream_t st = as_stream(stream);
+    float* lse = reinterpret_cast<float*>(region(ws, b.lse));
+    DUST_TRY(cuda_status(dust::launch_row_stats(Z, targets, T, V, lse, nullptr, st), "dust_head_bp_grad (row stats)"));
+    void* D = region(ws, b.d);
+    DUST_TRY(cuda_status(dust::launch_softmax_minus_onehot(Z, lse, targets, T, V, D, dt == DUST_BF16, st),
+                         "dust_head_bp_grad (softmax - onehot)"));
+    return run_gemm(b.plan, D, false, V, X, false, d_in, dt, V, d_in, T, G_bp, d_in, 0,
+                    reinterpret_cast<float*>(region(ws, b.part)), static_cast<uint32_t*>(ws), st);
+}
+
+size_t dust_cosine_workspace(void) { return dust::align_up(dust::kStatusBytes + dust::cosine_partial_bytes(), 256); }
+
+dust_status dust_cosine(const float* a, const float* b, long long n, double* out, void* ws, size_t ws_bytes,
+                        void* stream) {
+    DUST_REQUIRE(n > 0, DUST_ERR_INVALID_ARG, "n must be > 0");
+    DUST_TRY(check_ptr(a, "a"));
+    DUST_TRY(check_ptr(b, "b"));
+    DUST_TRY(check_ptr(out, "out"));
+    DUST_TRY(check_ptr(ws, "ws"));
+    DUST_REQUIRE(ws_bytes >= dust_cosine_workspace(), DUST_ERR_WORKSPACE, "workspace %zu bytes < %zu", ws_bytes,
+                 dust_cosine_workspace());
+    return cuda_status(dust::launch_cosine(a, b, n, reinterpret_cast<double*>(region(ws, dust::kStatusBytes)), out,
+                                           as_stream(stream)),
+                       "dust_cosine");
+}
+
 // ------------------------------------------------------------------ harness
 dust_status dust_noise_fill(dust_noise nz, uint32_t stream_id, int t0, int n_tok, int j0, int n_ch, float* out,
                             void* stream) {

@@ -65,6 +65,13 @@ cudaError_t run_toy_suffix(const float* Y, int T, int d, const int32_t* offs, in
                            const int32_t* targets, const dust_noise& nz, float* loss, float* c, void* ws,
                            cudaStream_t st);
 
+// cosine tuner support (tuner.cu)
+cudaError_t launch_softmax_minus_onehot(const float* Z, const float* lse, const int32_t* targets, int T, int V,
+                                        void* D, bool bf16, cudaStream_t stream);
+size_t cosine_partial_bytes();
+cudaError_t launch_cosine(const float* a, const float* b, long long n, double* part, double* out,
+                          cudaStream_t stream);
+
 // error reporting for entry points outside api.cu
 dust_status record_error(dust_status s, const char* msg);
 

@@ -70,6 +70,10 @@ _SIGS = {
     "dust_head_row_stats": ([_vp, _vp, _i, _i, _vp, _vp, _vp], _i),
     "dust_head_step": ([_vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _Noise, _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp], _i),
     "dust_head_step_workspace": ([_i, _i, _i, _i, _i, _i], _sz),
+    "dust_head_bp_grad": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp], _i),
+    "dust_head_bp_grad_workspace": ([_i, _i, _i, _i], _sz),
+    "dust_cosine": ([_vp, _vp, C.c_longlong, _vp, _vp, _sz, _vp], _i),
+    "dust_cosine_workspace": ([], _sz),
     "dust_noise_fill": ([_Noise, _u, _i, _i, _i, _i, _vp, _vp], _i),
     "dust_box_muller_words": ([_vp, _vp, C.c_longlong, _vp, _vp, _vp], _i),
     "dust_synth_costs": ([_vp, _i, _i, _Noise, _f, _vp, _vp], _i),
@@ -282,6 +286,32 @@ def head_step(targets: torch.Tensor, Vc: int, noise: Noise, *, Z: torch.Tensor |
                                 _dev(g_hat, "g_hat", torch.float32), _opt(g16, "g_hat_bf16"), _opt(G_W, "G_W"),
                                 int(bool(accumulate)), ws.data_ptr(), ws.numel(), _stream()))
     return {"g_hat": g_hat, "c": c, "g_hat_bf16": g16, "G_W": G_W}
+
+
+# ------------------------------------------------------------------ cosine tuner
+def head_bp_grad(Z: torch.Tensor, targets: torch.Tensor, X: torch.Tensor, G_bp: torch.Tensor | None = None):
+    """Backprop gradient of the head's summed cross entropy, sum_t (softmax(z_t) - e_y) x_t^T."""
+    T, V = Z.shape
+    d_in = X.shape[1]
+    dt = _dtype_code(X)
+    if G_bp is None:
+        G_bp = torch.empty(V, d_in, dtype=torch.float32, device=Z.device)
+    ws = workspace(lib().dust_head_bp_grad_workspace(T, d_in, V, dt), Z.device)
+    _check(lib().dust_head_bp_grad(_dev(Z, "Z", torch.float32), _dev(targets, "targets", torch.int32), _dev(X, "X"),
+                                   dt, T, d_in, V, _dev(G_bp, "G_bp", torch.float32), ws.data_ptr(), ws.numel(),
+                                   _stream()))
+    return G_bp
+
+
+def cosine(a: torch.Tensor, b: torch.Tensor) -> torch.Tensor:
+    """Device tensor of 4 doubles: (sum ab, sum aa, sum bb, cosine)."""
+    if a.numel() != b.numel():
+        raise ValueError("a and b must have the same number of elements")
+    out = torch.empty(4, dtype=torch.float64, device=a.device)
+    ws = workspace(lib().dust_cosine_workspace(), a.device)
+    _check(lib().dust_cosine(_dev(a, "a", torch.float32), _dev(b, "b", torch.float32), a.numel(), out.data_ptr(),
+                             ws.data_ptr(), ws.numel(), _stream()))
+    return out
 
 
 # ------------------------------------------------------------------ harness

@@ -1,0 +1,74 @@
+"""Choosing sigma by the cosine criterion, on the library's kernels.
+
+cnblogs Dust explainer, section "真正的工作量：压住干扰" (last paragraph): the
+cheap way to set sigma (and gamma) per layer type is to maximise, on a single
+batch, the cosine between the Dust estimate and the backprop gradient; a high
+single-batch cosine screens candidates, training decides.  Section
+"梯度是"长"出来的": the cosine grows with the population as
+cos(K) = c_max / sqrt(1 + c/K).
+
+This module only orchestrates calls of the C ABI (head steps over draw
+ranges, the head's closed-form backprop gradient, the device cosine); the
+two-parameter law is fitted on the host from the handful of cosines.
+With the literal sign of the error equation the estimate approaches
+-grad_W, so the cosines are taken against -G_bp.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import dust
+
+
+def _neg_cos(G_W: torch.Tensor, G_bp: torch.Tensor) -> float:
+    return float(dust.cosine(G_W, -G_bp)[3].item())
+
+
+def head_population_sweep(X: torch.Tensor, W: torch.Tensor, targets: torch.Tensor, Vc: int, Ks, sigma: float,
+                          seed: int = 0, layer: int = 0, Z: torch.Tensor | None = None):
+    """cos(G_W(K), -G_bp) for increasing populations K (one pass over the
+    largest K: the draws are added range by range with accumulate = 1; the
+    cosine does not depend on the 1/(K sigma) scale).  Returns (Ks, cosines)."""
+    Ks = sorted(int(k) for k in Ks)
+    if Z is None:
+        Z = dust.logits(X, W)
+    G_bp = dust.head_bp_grad(Z, targets, X)
+    K_max = Ks[-1]
+    g = None
+    coss, prev = [], 0
+    G_W = torch.empty(W.shape[0], X.shape[1], dtype=torch.float32, device=X.device)
+    g16 = torch.empty(Z.shape, dtype=torch.bfloat16, device=X.device) if X.dtype == torch.bfloat16 else None
+    for K in Ks:
+        nz = dust.Noise(seed, layer, prev, K - prev, K_max, sigma)
+        out = dust.head_step(targets, Vc, nz, Z=Z, g_hat=g, g_hat_bf16=g16, accumulate=g is not None)
+        g = out["g_hat"]
+        dust.weight_grad(g16 if g16 is not None else g, X, G_W=G_W)
+        coss.append(_neg_cos(G_W, G_bp))
+        prev = K
+    return np.array(Ks), np.array(coss)
+
+
+def head_sigma_sweep(X, W, targets, Vc: int, K: int, sigmas, seed: int = 0, layer: int = 0, Z=None):
+    """cos(G_W, -G_bp) at population K for each sigma; returns (sigmas, cosines, best sigma)."""
+    if Z is None:
+        Z = dust.logits(X, W)
+    G_bp = dust.head_bp_grad(Z, targets, X)
+    coss = []
+    for s in sigmas:
+        out = dust.head_step(targets, Vc, dust.Noise(seed, layer, 0, K, K, float(s)), Z=Z, X=X, want_G_W=True,
+                             want_bf16=X.dtype == torch.bfloat16)
+        coss.append(_neg_cos(out["G_W"], G_bp))
+    coss = np.array(coss)
+    return np.array(sigmas, dtype=float), coss, float(np.asarray(sigmas)[int(np.argmax(coss))])
+
+
+def fit_cosine_law(Ks, coss):
+    """Least-squares fit of cos(K) = c_max / sqrt(1 + c/K): with y = 1/cos^2,
+    y = (1 + c/K) / c_max^2 is linear in 1/K.  Returns (c_max, c)."""
+    Ks = np.asarray(Ks, dtype=float)
+    y = 1.0 / np.asarray(coss, dtype=float) ** 2
+    A = np.stack([np.ones_like(Ks), 1.0 / Ks], axis=1)
+    (a0, a1), *_ = np.linalg.lstsq(A, y, rcond=None)
+    c_max = 1.0 / np.sqrt(a0)
+    return float(c_max), float(a1 / a0)

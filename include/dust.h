@@ -202,6 +202,30 @@ dust_status dust_head_step(const void *X, const void *W, dust_dtype dt, const fl
                            void *stream);
 size_t dust_head_step_workspace(int T, int d_in, int V, dust_dtype dt, int has_Z, int want_G_W);
 
+/* ------------------------------------------------------------------ cosine tuner
+ * cnblogs Dust explainer, section "真正的工作量：压住干扰" (last paragraph): the
+ * hyper-parameters can be chosen by maximising, on one batch, the cosine
+ * between the Dust estimate and the backprop gradient; section
+ * "梯度是"长"出来的": cos(K) = c_max / sqrt(1 + c/K).
+ *
+ * Backprop gradient of the head's summed cross entropy on cached logits:
+ * G_bp[v][i] = sum_t (softmax(Z_t)[v] - [v == y_t]) X[t][i]  ([V][d_in] fp32).
+ * With the literal sign of the error equation the Dust head estimate
+ * approaches -G_bp.  X: [T][d_in] of dtype dt (bf16: tensor cores, the
+ * softmax difference rounded to bf16; f32: CUDA cores).  Workspace:
+ * dust_head_bp_grad_workspace(). */
+dust_status dust_head_bp_grad(const float *Z, const int32_t *targets, const void *X, dust_dtype dt,
+                              int T, int d_in, int V, float *G_bp, void *ws, size_t ws_bytes,
+                              void *stream);
+size_t dust_head_bp_grad_workspace(int T, int d_in, int V, dust_dtype dt);
+
+/* out (device, 4 doubles) = { sum a b, sum a a, sum b b, cosine } over n fp32
+ * elements, accumulated in double in a fixed order (deterministic).
+ * Workspace: dust_cosine_workspace(). */
+dust_status dust_cosine(const float *a, const float *b, long long n, double *out, void *ws,
+                        size_t ws_bytes, void *stream);
+size_t dust_cosine_workspace(void);
+
 /* ------------------------------------------------------------------ harness / debug
  * Noise: out[k][t][j] = a(seed, layer, draw_begin + k, t0 + t, j0 + j) from
  * Philox stream `stream_id` (0: activation noise, 1: synthetic observation

@@ -67,6 +67,10 @@ def lib():
         L.orc_head_step.argtypes = [_f32p, _i32p, _i32p, i32, i32, i32, u32, u32, u32, i32,
                                     i32, dbl, _nullable(_f64p), _f64p]
         L.orc_head_step.restype = i32
+        L.orc_head_bp_grad.argtypes = [_f32p, _i32p, _f32p, i32, i32, i32, _i32p, i32, _f64p]
+        L.orc_head_bp_grad.restype = i32
+        L.orc_cosine.argtypes = [_f32p, _f32p, C.c_longlong]
+        L.orc_cosine.restype = dbl
         L.orc_synth_costs.argtypes = [_f32p, i32, i32, u32, u32, dbl, dbl, _i32p, _i32p, i32, _f64p]
         L.orc_synth_costs.restype = i32
         L.orc_toy_suffix_losses.argtypes = [_f32p, _f32p, i32, i32, i32, _i32p, i32,
@@ -240,6 +244,24 @@ def head_step(Zrows, y, toks, Vc, seed, layer, draw_begin, nd, K_total, sigma, w
     _check(lib().orc_head_step(Zrows, _i32(y), _i32(toks), n, V, Vc, seed, layer, draw_begin,
                                nd, K_total, float(sigma), c, g), "head_step")
     return c, g
+
+
+def head_bp_grad(Z, y, X, rows=None) -> np.ndarray:
+    """Backprop gradient of sum_t CE(z_t, y_t) w.r.t. W (rows of [V][d_in]), float64."""
+    Z = _f32(Z)
+    X = _f32(X)
+    T, V = Z.shape
+    d_in = X.shape[1]
+    rows = _i32(np.arange(V) if rows is None else rows)
+    G = np.zeros((len(rows), d_in), np.float64)
+    _check(lib().orc_head_bp_grad(Z, _i32(y), X, T, d_in, V, rows, len(rows), G), "head_bp_grad")
+    return G
+
+
+def cosine(a, b) -> float:
+    a = _f32(np.ravel(a))
+    b = _f32(np.ravel(b))
+    return float(lib().orc_cosine(a, b, a.size))
 
 
 # ---------------------------------------------------------------- toy suffix

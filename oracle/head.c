@@ -106,3 +106,42 @@ int orc_head_step(const float *Zrows, const int32_t *y, const int32_t *toks,
     }
     return err;
 }
+
+/* Backprop gradient of sum_t l_t with respect to W for the listed output rows:
+ * G[n][i] = sum_t (softmax(z_t)[rows[n]] - [rows[n] == y_t]) X[t][i]. */
+int orc_head_bp_grad(const float *Z, const int32_t *y, const float *X, int T, int d_in, int V,
+                     const int32_t *rows, int n_rows, double *G)
+{
+    double *lse = (double *)malloc(sizeof(double) * (size_t)T);
+    double *zt = (double *)malloc(sizeof(double) * (size_t)V);
+    if (!lse || !zt) { free(lse); free(zt); return -1; }
+    for (int t = 0; t < T; ++t) {
+        for (int v = 0; v < V; ++v) zt[v] = (double)Z[(size_t)t * V + v];
+        lse[t] = logsumexp(zt, V);
+    }
+    free(zt);
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < n_rows; ++n) {
+        const int v = rows[n];
+        double *Gn = G + (size_t)n * d_in;
+        for (int i = 0; i < d_in; ++i) Gn[i] = 0.0;
+        for (int t = 0; t < T; ++t) {
+            const double d = exp((double)Z[(size_t)t * V + v] - lse[t]) - (y[t] == v ? 1.0 : 0.0);
+            for (int i = 0; i < d_in; ++i) Gn[i] += d * (double)X[(size_t)t * d_in + i];
+        }
+    }
+    free(lse);
+    return 0;
+}
+
+/* Cosine similarity of two vectors, accumulated in double. */
+double orc_cosine(const float *a, const float *b, long long n)
+{
+    double ab = 0.0, aa = 0.0, bb = 0.0;
+    for (long long i = 0; i < n; ++i) {
+        ab += (double)a[i] * (double)b[i];
+        aa += (double)a[i] * (double)a[i];
+        bb += (double)b[i] * (double)b[i];
+    }
+    return ab / (sqrt(aa) * sqrt(bb));
+}

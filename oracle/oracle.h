@@ -118,6 +118,14 @@ int orc_head_step(const float *Zrows, const int32_t *y, const int32_t *toks,
                   uint32_t draw_begin, int nd, int K_total, double sigma,
                   double *c, double *g);
 
+/* Backprop gradient of the head's summed cross entropy, rows of [V][d_in]:
+ * G[n][i] = sum_t (softmax(z_t)[rows[n]] - [rows[n] == y_t]) X[t][i]. */
+int orc_head_bp_grad(const float *Z, const int32_t *y, const float *X, int T, int d_in, int V,
+                     const int32_t *rows, int n_rows, double *G);
+
+/* Cosine similarity in double. */
+double orc_cosine(const float *a, const float *b, long long n);
+
 /* ---------------- synthetic costs (estimator-only workloads) ---------------- */
 
 /* c = sigma <u_s, a_s^(i)> + eps_scale * eps(i, s),

@@ -299,3 +299,35 @@ def test_suffix_clean_losses_and_small_sigma_linearity(orc):
         l1 = orc.toy_suffix_losses(X1, p["W"], np.array([0, 1], np.int32), p["Wq"], p["Wk"], p["Wv"],
                                    p["Wo"], p["Wout"], p["y"][t0:t0 + 1], 0, 1, 0.0, [0])
         np.testing.assert_allclose(l1[0, 0], clean[0, t0], rtol=1e-13)
+
+
+# ------------------------------------------------------------------ cosine tuner support
+
+def test_head_bp_grad_equals_autograd(orc):
+    """The head's backprop gradient (comparator of the cosine criterion)
+    against torch autograd in float64 (a library routine)."""
+    T, d, V = 30, 7, 11
+    X = I.normal((T, d), 1.0, seed=30)
+    W = I.normal((V, d), 0.5, seed=31)
+    y = I.targets(T, V, seed=32)
+    Wt = torch.tensor(W, dtype=torch.float64, requires_grad=True)
+    Z = torch.tensor(X, dtype=torch.float64) @ Wt.T
+    torch.nn.functional.cross_entropy(Z, torch.tensor(y, dtype=torch.int64), reduction="sum").backward()
+    Zf = (X.astype(np.float64) @ W.astype(np.float64).T).astype(np.float32)
+    G = orc.head_bp_grad(Zf, y, X)
+    np.testing.assert_allclose(G, Wt.grad.numpy(), rtol=1e-5, atol=1e-5 * np.abs(Wt.grad.numpy()).max())
+
+
+def test_cosine_equals_numpy(orc):
+    a = I.normal(1000, 1.0, seed=33)
+    b = I.normal(1000, 1.0, seed=34) + 0.5 * a
+    ref = float(np.dot(a.astype(np.float64), b) / (np.linalg.norm(a.astype(np.float64)) * np.linalg.norm(b.astype(np.float64))))
+    assert abs(orc.cosine(a, b) - ref) < 1e-12
+
+
+def test_cosine_law_fit_recovers_parameters():
+    from activation_perturbation_es_b200 import tuner
+    Ks = np.array([64, 128, 256, 1024, 4096, 16384])
+    c_max, c = 0.93, 850.0
+    cm, cc = tuner.fit_cosine_law(Ks, c_max / np.sqrt(1 + c / Ks))
+    assert abs(cm - c_max) < 1e-9 and abs(cc - c) < 1e-6
