@@ -181,11 +181,36 @@ dust_status dust_reward_scan(const float* c, float* r, int K, int T, const int32
                        "dust_reward_scan");
 }
 
+size_t dust_reward_scan_split_workspace(int K, int T) {
+    Layout L;
+    if (K > 0 && T > 0) L.add(dust::reward_scan_chunks_workspace(K, T));
+    return L.off;
+}
+
+dust_status dust_reward_scan_split(const float* c, float* r, int K, int T, const int32_t* seq_offsets, int n_seq,
+                                   float gamma, void* ws, size_t ws_bytes, void* stream) {
+    DUST_REQUIRE(K > 0 && T > 0, DUST_ERR_INVALID_ARG, "K and T must be > 0 (K=%d, T=%d)", K, T);
+    DUST_REQUIRE(std::isfinite(gamma) && gamma >= 0.0f && gamma <= 1.0f, DUST_ERR_INVALID_ARG,
+                 "gamma must be in [0, 1]");
+    DUST_TRY(check_ptr(c, "c"));
+    DUST_TRY(check_ptr(r, "r"));
+    DUST_TRY(check_seq(seq_offsets, n_seq, K, T));
+    DUST_TRY(check_ptr(ws, "ws"));
+    const size_t need = dust_reward_scan_split_workspace(K, T);
+    DUST_REQUIRE(ws_bytes >= need, DUST_ERR_WORKSPACE, "workspace %zu bytes < %zu", ws_bytes, need);
+    return cuda_status(dust::launch_reward_scan_chunks(c, r, K, T, seq_offsets, n_seq, gamma,
+                                                       region(ws, dust::kStatusBytes), as_stream(stream)),
+                       "dust_reward_scan_split");
+}
+
 // ------------------------------------------------------------------ a5
 size_t dust_layer_estimate_workspace(int draw_count, int T, int d_out, int is_r, float gamma) {
     (void)d_out;
     Layout L;
-    if (!is_r && gamma != 0.0f && draw_count > 0 && T > 0) L.add(sizeof(float) * static_cast<size_t>(draw_count) * T);
+    if (!is_r && gamma != 0.0f && draw_count > 0 && T > 0) {
+        L.add(sizeof(float) * static_cast<size_t>(draw_count) * T);          // r
+        L.add(dust::reward_scan_chunks_workspace(draw_count, T));             // chunked scan (few long sequences)
+    }
     return L.off;
 }
 
@@ -208,10 +233,14 @@ dust_status dust_layer_estimate(const float* c_or_r, int is_r, int T, int d_out,
     cudaStream_t st = as_stream(stream);
     const float* r = c_or_r;
     if (need_scan) {
+        const int K = static_cast<int>(nz.draw_count);
         float* rw = reinterpret_cast<float*>(region(ws, dust::kStatusBytes));
-        DUST_TRY(cuda_status(dust::launch_reward_scan(c_or_r, rw, static_cast<int>(nz.draw_count), T, seq_offsets,
-                                                      n_seq, gamma, st),
-                             "dust_layer_estimate (scan)"));
+        const size_t chunk_off = dust::align_up(dust::kStatusBytes + sizeof(float) * static_cast<size_t>(K) * T, 256);
+        const cudaError_t e = dust::reward_scan_prefers_chunks(K, T, n_seq)
+                                  ? dust::launch_reward_scan_chunks(c_or_r, rw, K, T, seq_offsets, n_seq, gamma,
+                                                                    region(ws, chunk_off), st)
+                                  : dust::launch_reward_scan(c_or_r, rw, K, T, seq_offsets, n_seq, gamma, st);
+        DUST_TRY(cuda_status(e, "dust_layer_estimate (scan)"));
         r = rw;
     }
     return cuda_status(dust::launch_layer_estimate(r, T, d_out, nz, g_hat, g_hat_bf16, accumulate, st),

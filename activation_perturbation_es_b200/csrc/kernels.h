@@ -15,6 +15,13 @@ namespace dust {
 cudaError_t launch_reward_scan(const float* c, float* r, int K, int T, const int32_t* offs,
                                int n_seq, float gamma, cudaStream_t stream);
 
+// a4 for few long sequences: chunked three-pass scan; scratch holds
+// reward_scan_chunks_workspace(K, T) bytes (chunk maps and carries)
+size_t reward_scan_chunks_workspace(int K, int T);
+bool reward_scan_prefers_chunks(int K, int T, int n_seq);
+cudaError_t launch_reward_scan_chunks(const float* c, float* r, int K, int T, const int32_t* offs, int n_seq,
+                                      float gamma, void* scratch, cudaStream_t stream);
+
 // a1 + a5 (layer_estimate.cu): g (+)= scale * sum_k r[k][t] a(draw_begin + k, t, j)
 cudaError_t launch_layer_estimate(const float* r, int T, int d_out, const dust_noise& nz,
                                   float* g, void* g_bf16, int accumulate, cudaStream_t stream);

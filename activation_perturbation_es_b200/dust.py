@@ -60,6 +60,8 @@ _SIGS = {
     "dust_poll_status": ([_vp, _vp], _i),
     "dust_selftest_bounded_wait": ([_vp, _u, _vp], _i),
     "dust_reward_scan": ([_vp, _vp, _i, _i, _vp, _i, _f, _vp], _i),
+    "dust_reward_scan_split": ([_vp, _vp, _i, _i, _vp, _i, _f, _vp, _sz, _vp], _i),
+    "dust_reward_scan_split_workspace": ([_i, _i], _sz),
     "dust_layer_estimate": ([_vp, _i, _i, _i, _vp, _i, _f, _Noise, _vp, _vp, _i, _vp, _sz, _vp], _i),
     "dust_layer_estimate_workspace": ([_i, _i, _i, _i, _f], _sz),
     "dust_layer_estimate_noalloc": ([_vp, _i, _i, _vp, _i, _f, _Noise, _vp, _vp, _i, _vp], _i),
@@ -165,6 +167,17 @@ def reward_scan(c: torch.Tensor, seq_offsets: torch.Tensor, gamma: float, out: t
     _check(lib().dust_reward_scan(_dev(c, "c", torch.float32), _dev(r, "r", torch.float32), K, T,
                                   _dev(seq_offsets, "seq_offsets", torch.int32), seq_offsets.numel() - 1,
                                   float(gamma), _stream()))
+    return r
+
+
+def reward_scan_split(c: torch.Tensor, seq_offsets: torch.Tensor, gamma: float, out: torch.Tensor | None = None):
+    """dust_reward_scan_split: the reward scan over 1024-token chunks (for few long sequences)."""
+    K, T = c.shape
+    r = torch.empty_like(c) if out is None else out
+    ws = workspace(lib().dust_reward_scan_split_workspace(K, T), c.device)
+    _check(lib().dust_reward_scan_split(_dev(c, "c", torch.float32), _dev(r, "r", torch.float32), K, T,
+                                        _dev(seq_offsets, "seq_offsets", torch.int32), seq_offsets.numel() - 1,
+                                        float(gamma), ws.data_ptr(), ws.numel(), _stream()))
     return r
 
 

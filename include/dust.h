@@ -107,6 +107,17 @@ dust_status dust_reward_scan(const float *c, float *r, int K, int T,
                              const int32_t *seq_offsets, int n_seq, float gamma,
                              void *stream);
 
+/* Same result as dust_reward_scan, computed over fixed 1024-token chunks of
+ * every draw row in parallel (the chunk maps x -> c + g x are composed per
+ * chunk, the carries between chunks resolved in a second step, then every
+ * chunk rescanned with its carry).  For few, long sequences, where the
+ * per-sequence scan has too few blocks to fill the GPU.  Reads c twice.
+ * r may alias c.  Workspace: dust_reward_scan_split_workspace(). */
+dust_status dust_reward_scan_split(const float *c, float *r, int K, int T,
+                                   const int32_t *seq_offsets, int n_seq, float gamma,
+                                   void *ws, size_t ws_bytes, void *stream);
+size_t dust_reward_scan_split_workspace(int K, int T);
+
 /* ------------------------------------------------------------------ a5: error
  * [CA, error equation] g_hat[t][j] (+)= -(1/(K_total sigma))
  *     sum_{k < draw_count} r[k][t] a(seed, layer, draw_begin + k, t, j).

@@ -90,6 +90,44 @@ def test_reward_scan_parity(orc, lengths, K, gamma):
     np.testing.assert_array_equal(host(inplace).view(np.uint32), r.view(np.uint32))
 
 
+SPLIT_CASES = [
+    ([70000], 3),                                   # one long sequence (69 chunks)
+    ([1500, 1, 0, 2047, 1024, 3000, 5], 4),         # boundaries inside and at chunk edges, empty sequences
+    ([5, 0, 1, 17, 3, 0, 33, 2], 7),                # many sequences inside one chunk
+    ([1], 2),
+]
+
+
+@pytest.mark.parametrize("lengths,K", SPLIT_CASES)
+@pytest.mark.parametrize("gamma", [0.0, 0.5, 0.99, 1.0])
+def test_reward_scan_split_parity(orc, lengths, K, gamma):
+    """The chunked scan gives the same rewards as the oracle's recurrence (and the
+    per-sequence scan), in place too."""
+    off = I.offsets_from_lengths(lengths)
+    T = int(off[-1])
+    c = I.normal((K, T), 0.01, seed=K + T + 1)
+    ref = orc.reward_scan(c, off, gamma)
+    gc, goff = cu(c), cu(off)
+    r = host(dust.reward_scan_split(gc, goff, gamma))
+    assert rel_err(r, ref) < 1e-5
+    if gamma == 0.0:
+        np.testing.assert_array_equal(r.view(np.uint32), c.view(np.uint32))
+    inplace = gc.clone()
+    dust.reward_scan_split(inplace, goff, gamma, out=inplace)
+    np.testing.assert_array_equal(host(inplace).view(np.uint32), r.view(np.uint32))
+
+
+def test_layer_estimate_long_sequence_uses_chunked_scan(orc):
+    """K x n_seq small and one long sequence: the estimate runs the chunked scan internally."""
+    T, K, d = 9000, 4, 16
+    off = np.array([0, T], np.int32)
+    c = I.normal((K, T), 0.01, seed=77)
+    g, _ = dust.layer_estimate(cu(c), False, cu(off), 0.97, dust.Noise(2, 3, 0, K, K, 0.01), d)
+    toks = np.array([0, 1023, 1024, 4500, 8999])
+    ref = orc.layer_estimate(c, False, d, off, 0.97, 2, 3, 0, K, 0.01, toks)
+    assert rel_err(host(g)[toks], ref) < 1e-5
+
+
 # ------------------------------------------------------------------ a5 estimate
 @pytest.mark.parametrize("T,d_out,K,gamma,is_r", [
     (37, 10, 9, 0.9, False),
