@@ -333,13 +333,15 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32 (noise, CE, reduction); bf16 in / f32 acc (tcgen05 GEMMs)",
+            "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded; inputs > L2, no flush needed)",
             "config": {"workload": w.name, "tokens_per_rank": w.T, "n_seq": w.n_seq, "seq_len": w.seq_len,
                        "draws": K, "sigma": w.sigma, "gamma_hidden": w.gamma,
                        "hidden": [[h.d_in, h.d_out] for h in w.hidden],
                        "head": {"d": w.head_d, "V": w.V, "Vc": w.Vc} if w.V else None,
-                       "parallelism": f"dp{world}", "l2": "inputs larger than L2 (126 MB); no flush"},
+                       "parallelism": f"dp{world}", "l2": "inputs larger than L2 (126 MB); no flush",
+                       "arithmetic": "f32 noise, cross entropy and reductions; bf16 GEMM operands with f32 "
+                                     "accumulation in TMEM (tcgen05)"},
             "roofline": {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
             | {"kernel": dominant["name"], "clock_mhz_for_peak": dominant.get("clock_mhz_for_peak"),
                "peak_source": dominant.get("peak_source")},
