@@ -77,6 +77,9 @@ def lib():
                                             _f32p, _f32p, _f32p, _f32p, i32, _f32p, i32,
                                             _i32p, u32, u32, dbl, i32, _i32p, i32, _f64p]
         L.orc_toy_suffix_losses.restype = i32
+        L.orc_attention_internal_costs.argtypes = [_f32p, i32, i32, _i32p, i32, _f32p, _f32p, _f32p, _f32p, i32, i32,
+                                                   _f32p, u32, u32, dbl, _i32p, i32, _f64p]
+        L.orc_attention_internal_costs.restype = i32
         _lib = L
     return _lib
 
@@ -281,3 +284,19 @@ def toy_suffix_losses(X, W, seq_offsets, Wq, Wk, Wv, Wo, Wout, targets, seed, la
                                        int(bool(with_noise)), draws, len(draws), loss),
            "toy_suffix_losses")
     return loss
+
+
+# ---------------------------------------------------------------- attention-internal scoring
+
+def attention_internal_costs(Y, seq_offsets, Wq, Wk, Wv, Wo, which, G, seed, layer, sigma, draws) -> np.ndarray:
+    """c[n][t] = -<z~_t - z_t, G_t> for perturbations of projection `which` (0 q, 1 k, 2 v)."""
+    Y, Wq, Wk, Wv, Wo, G = (_f32(a) for a in (Y, Wq, Wk, Wv, Wo, G))
+    T, d = Y.shape
+    dh = Wq.shape[0]
+    off = _i32(seq_offsets)
+    draws = _i32(draws)
+    c = np.zeros((len(draws), T), np.float64)
+    _check(lib().orc_attention_internal_costs(Y, T, d, off, len(off) - 1, Wq, Wk, Wv, Wo, dh, int(which), G,
+                                              seed, layer, float(sigma), draws, len(draws), c),
+           "attention_internal_costs")
+    return c

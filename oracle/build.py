@@ -12,7 +12,7 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SOURCES = ["noise.c", "estimator.c", "head.c", "suffix.c"]
+SOURCES = ["noise.c", "estimator.c", "head.c", "suffix.c", "attention.c"]
 LIB = os.path.join(HERE, "liboracle.so")
 
 

@@ -151,6 +151,16 @@ int orc_toy_suffix_losses(const float *X, const float *W, int T, int d_in, int d
                           double sigma, int with_noise,
                           const int32_t *draws, int nd, double *loss);
 
+/* ---------------- attention-internal scoring ---------------- */
+
+/* c[n][t] = -< z~_t - z_t, G_t > where z = Attn(Y Wq^T, Y Wk^T, Y Wv^T) Wo^T and
+ * z~ has sigma a(draws[n]) added to projection `which` (0 = q, 1 = k, 2 = v;
+ * channel = projection channel).  Y, G: [T][d]; Wq, Wk, Wv: [dh][d]; Wo: [d][dh]. */
+int orc_attention_internal_costs(const float *Y, int T, int d, const int32_t *offs, int n_seq,
+                                 const float *Wq, const float *Wk, const float *Wv, const float *Wo,
+                                 int dh, int which, const float *G, uint32_t seed, uint32_t layer,
+                                 double sigma, const int32_t *draws, int nd, double *c);
+
 #ifdef __cplusplus
 }
 #endif

@@ -331,3 +331,72 @@ def test_cosine_law_fit_recovers_parameters():
     c_max, c = 0.93, 850.0
     cm, cc = tuner.fit_cosine_law(Ks, c_max / np.sqrt(1 + c / Ks))
     assert abs(cm - c_max) < 1e-9 and abs(cc - c) < 1e-6
+
+
+# ------------------------------------------------------------------ attention-internal scoring
+
+def _attn_small(seed=40, T=14, d=8, dh=4):
+    r = np.random.Generator(np.random.PCG64(seed))
+    f = lambda *s: r.standard_normal(s).astype(np.float32) * np.float32(0.5)
+    return dict(Y=f(T, d), Wq=f(dh, d), Wk=f(dh, d), Wv=f(dh, d), Wo=f(d, dh), G=f(T, d),
+                off=np.array([0, 6, 6, T], np.int32))
+
+
+def test_attention_costs_zero_when_the_projection_cannot_matter(orc):
+    """q has no effect when Wk = 0 (every score is 0), k none when Wq = 0."""
+    p = _attn_small()
+    args = lambda P, which: (P["Y"], P["off"], P["Wq"], P["Wk"], P["Wv"], P["Wo"], which, P["G"], 0, 5, 0.1, [0, 3])
+    pq = dict(p, Wk=np.zeros_like(p["Wk"]))
+    assert np.all(orc.attention_internal_costs(*args(pq, 0)) == 0.0)
+    pk = dict(p, Wq=np.zeros_like(p["Wq"]))
+    assert np.all(orc.attention_internal_costs(*args(pk, 1)) == 0.0)
+    # but the value projection matters in both cases
+    assert np.any(orc.attention_internal_costs(*args(pq, 2)) != 0.0)
+
+
+def test_attention_costs_uniform_attention_closed_form(orc):
+    """Wq = Wk = 0: attention is the causal running mean, so a value perturbation
+    changes the output by (running mean of sigma a) Wo^T (numpy cumsum)."""
+    p = _attn_small()
+    p["Wq"] = np.zeros_like(p["Wq"])
+    p["Wk"] = np.zeros_like(p["Wk"])
+    sigma, T, dh = 0.1, p["Y"].shape[0], p["Wq"].shape[0]
+    c = orc.attention_internal_costs(p["Y"], p["off"], p["Wq"], p["Wk"], p["Wv"], p["Wo"], 2, p["G"], 0, 5, sigma, [2])
+    a = orc.noise_block(0, 5, 2, 1, np.arange(T), 0, dh)[0].astype(np.float64)
+    dz = np.zeros((T, p["Y"].shape[1]))
+    off = p["off"]
+    for q in range(len(off) - 1):
+        seg = a[off[q]:off[q + 1]]
+        if len(seg):
+            m = np.cumsum(seg, axis=0) / np.arange(1, len(seg) + 1)[:, None]
+            dz[off[q]:off[q + 1]] = sigma * m @ p["Wo"].astype(np.float64).T
+    np.testing.assert_allclose(c[0], -np.sum(dz * p["G"], axis=1), rtol=1e-10, atol=1e-14)
+
+
+def test_attention_value_estimate_converges_to_backprop_through_uniform_attention(orc):
+    """With uniform attention the value-projection costs are linear in the noise,
+    and with gamma = 1 the estimate's expectation is exactly the backprop of
+    <z, g> to v_t: E[g_hat_t] = sum_{s >= t, same seq} (G_s Wo) / n_s, n_s the
+    size of s's causal prefix.  The error falls like K^-1/2."""
+    p = _attn_small(seed=41, T=10, d=6, dh=8)
+    p["Wq"] = np.zeros_like(p["Wq"])
+    p["Wk"] = np.zeros_like(p["Wk"])
+    off = np.array([0, 4, 10], np.int32)
+    T, dh, sigma = 10, 8, 0.05
+    target = np.zeros((T, dh))
+    w = p["G"].astype(np.float64) @ p["Wo"].astype(np.float64)       # G_s Wo
+    for q in range(2):
+        for t in range(off[q], off[q + 1]):
+            for s in range(t, off[q + 1]):
+                target[t] += w[s] / (s - off[q] + 1)
+    Kmax = 8192
+    c = orc.attention_internal_costs(p["Y"], off, p["Wq"], p["Wk"], p["Wv"], p["Wo"], 2, p["G"], 1, 7, sigma,
+                                     np.arange(Kmax)).astype(np.float32)
+    errs = []
+    Ks = [128, 512, 2048, 8192]
+    for K in Ks:
+        g = orc.layer_estimate(c[:K], False, dh, off, 1.0, 1, 7, 0, K, sigma, np.arange(T))
+        errs.append(np.linalg.norm(g - target) / np.linalg.norm(target))
+    slope = np.polyfit(np.log(Ks), np.log(errs), 1)[0]
+    assert -0.6 <= slope <= -0.4, (slope, errs)
+    assert errs[-1] < 0.2, errs
