@@ -507,4 +507,28 @@ dust_status dust_toy_suffix_losses(const float* Y, int T, int d, const int32_t* 
                        "dust_toy_suffix_losses");
 }
 
+size_t dust_attention_internal_costs_workspace(int draw_count, int T, int d, int dh) {
+    if (draw_count <= 0 || T <= 0 || d <= 0 || dh <= 0) return dust::kStatusBytes;
+    return dust::attention_scoring_workspace_bytes(draw_count, T, d, dh);
+}
+
+dust_status dust_attention_internal_costs(const float* Y, int T, int d, const int32_t* seq_offsets, int n_seq,
+                                          const float* Wq, const float* Wk, const float* Wv, const float* Wo, int dh,
+                                          int which, const float* G, dust_noise nz, float* c, void* ws,
+                                          size_t ws_bytes, void* stream) {
+    DUST_TRY(check_noise(nz));
+    DUST_REQUIRE(T > 0 && d > 0 && dh > 0, DUST_ERR_INVALID_ARG, "T, d, dh must be > 0");
+    DUST_REQUIRE(which >= 0 && which <= 2, DUST_ERR_INVALID_ARG, "which must be 0 (q), 1 (k) or 2 (v)");
+    DUST_REQUIRE(dh % 4 == 0 && dh <= 128, DUST_ERR_UNSUPPORTED, "attention scoring supports dh %% 4 == 0, dh <= 128");
+    DUST_TRY(check_seq(seq_offsets, n_seq, 1, T));
+    const void* ptrs[] = {Y, Wq, Wk, Wv, Wo, G, c, ws};
+    const char* names[] = {"Y", "Wq", "Wk", "Wv", "Wo", "G", "c", "ws"};
+    for (int i = 0; i < 8; ++i) DUST_TRY(check_ptr(ptrs[i], names[i]));
+    const size_t need = dust_attention_internal_costs_workspace(static_cast<int>(nz.draw_count), T, d, dh);
+    DUST_REQUIRE(ws_bytes >= need, DUST_ERR_WORKSPACE, "workspace %zu bytes < %zu", ws_bytes, need);
+    return cuda_status(dust::run_attention_internal_costs(Y, T, d, seq_offsets, n_seq, Wq, Wk, Wv, Wo, dh, which, G,
+                                                          nz, c, ws, as_stream(stream)),
+                       "dust_attention_internal_costs");
+}
+
 }  // extern "C"

@@ -82,6 +82,19 @@ cudaError_t launch_cosine(const float* a, const float* b, long long n, double* p
 // error reporting for entry points outside api.cu
 dust_status record_error(dust_status s, const char* msg);
 
+// causal softmax attention per sequence (toy_suffix.cu); q, k, v [nb][T][dh]
+// with batch strides in elements (0: shared by the batch), o [nb][T][dh]
+cudaError_t launch_causal_attention(const float* q, const float* k, const float* v, long long q_bs, long long k_bs,
+                                    long long v_bs, int nb, int T, int dh, const int32_t* offs, int n_seq,
+                                    float* o, cudaStream_t stream);
+
+// attention-internal scoring (attention_scoring.cu)
+size_t attention_scoring_workspace_bytes(int draw_count, int T, int d, int dh);
+cudaError_t run_attention_internal_costs(const float* Y, int T, int d, const int32_t* offs, int n_seq,
+                                         const float* Wq, const float* Wk, const float* Wv, const float* Wo, int dh,
+                                         int which, const float* G, const dust_noise& nz, float* c, void* ws,
+                                         cudaStream_t st);
+
 // fp32 -> bf16 (RNE) copy
 cudaError_t launch_to_bf16(const float* src, void* dst, size_t n, cudaStream_t stream);
 

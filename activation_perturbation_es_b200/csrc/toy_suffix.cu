@@ -43,29 +43,33 @@ __global__ void perturb_kernel(const float* __restrict__ Y, int T, int d, uint32
 
 // One warp per (batch row, token): online softmax over the token's causal
 // prefix inside its sequence, in chunks of 32 keys (one key per lane).
+// q, k, v are [nb][T][dh] with a batch stride each (0: shared by the batch).
 __global__ void __launch_bounds__(256)
-causal_attention_kernel(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
-                        int nb, int T, int dh, const int32_t* __restrict__ offs, int n_seq, float scale,
-                        float* __restrict__ o) {
+causal_attention_kernel(const float* __restrict__ qa, const float* __restrict__ ka, const float* __restrict__ va,
+                        long long q_bs, long long k_bs, long long v_bs, int nb, int T, int dh,
+                        const int32_t* __restrict__ offs, int n_seq, float scale, float* __restrict__ o) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long row = blockIdx.x * 8LL + warp;
     if (row >= static_cast<long long>(nb) * T) return;
     const int t = static_cast<int>(row % T);
-    const long long base = row - t;   // first row of this batch entry
+    const long long b = row / T;
+    const float* q = qa + b * q_bs;
+    const float* k = ka + b * k_bs;
+    const float* v = va + b * v_bs;
     // sequence of t (offsets clamped; linear search is fine for a harness)
     int s0 = 0;
     for (int sq = 0; sq < n_seq; ++sq) {
         const int2 sb = seq_bounds(offs, sq, T);
         if (t >= sb.x && t < sb.y) { s0 = sb.x; break; }
     }
-    const float* qt = q + row * dh;
+    const float* qt = q + static_cast<long long>(t) * dh;
     float m = -INFINITY, l = 0.0f;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};   // channels lane + 32 e, dh <= 128
     for (int u0 = s0; u0 <= t; u0 += 32) {
         const int u = u0 + lane;
         float sc = -INFINITY;
         if (u <= t) {
-            const float* ku = k + (base + u) * dh;
+            const float* ku = k + static_cast<long long>(u) * dh;
             float s = 0.0f;
             for (int e = 0; e < dh; ++e) s = fmaf(__ldg(qt + e), __ldg(ku + e), s);
             sc = s * scale;
@@ -80,7 +84,7 @@ causal_attention_kernel(const float* __restrict__ q, const float* __restrict__ k
         const int n_keys = min(32, t - u0 + 1);
         for (int j = 0; j < n_keys; ++j) {
             const float pj = __shfl_sync(0xffffffffu, p, j);
-            const float* vu = v + (base + u0 + j) * dh;
+            const float* vu = v + static_cast<long long>(u0 + j) * dh;
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 if (lane + 32 * e < dh) acc[e] = fmaf(pj, __ldg(vu + lane + 32 * e), acc[e]);
@@ -115,6 +119,19 @@ __global__ void diff_kernel(const float* __restrict__ loss, long long n, int T, 
          i += static_cast<long long>(gridDim.x) * blockDim.x)
         c[i] = loss[T + i] - loss[i % T];
 }
+
+}  // namespace
+
+cudaError_t launch_causal_attention(const float* q, const float* k, const float* v, long long q_bs, long long k_bs,
+                                    long long v_bs, int nb, int T, int dh, const int32_t* offs, int n_seq,
+                                    float* o, cudaStream_t stream) {
+    const long long rows = static_cast<long long>(nb) * T;
+    causal_attention_kernel<<<static_cast<unsigned>(ceil_div(rows, 8)), 256, 0, stream>>>(
+        q, k, v, q_bs, k_bs, v_bs, nb, T, dh, offs, n_seq, 1.0f / std::sqrt(static_cast<float>(dh)), o);
+    return cudaGetLastError();
+}
+
+namespace {
 
 unsigned blocks_for(long long n, int per) {
     const long long b = ceil_div(n, per);
@@ -192,9 +209,8 @@ cudaError_t run_toy_suffix(const float* Y, int T, int d, const int32_t* offs, in
             e = launch_gemm_simt(yt, true, d, Ws[w], true, d, DUST_F32, M, dh, d, outs[w], dh, 0, part,
                                  gemm_simt_splits(M, dh, d), st);
         if (e != cudaSuccess) break;
-        causal_attention_kernel<<<static_cast<unsigned>(ceil_div(rows, 8)), 256, 0, st>>>(
-            q, k, v, nb, T, dh, offs, n_seq, 1.0f / std::sqrt(static_cast<float>(dh)), o);
-        if ((e = cudaGetLastError()) != cudaSuccess) break;
+        const long long bs = static_cast<long long>(T) * dh;
+        if ((e = launch_causal_attention(q, k, v, bs, bs, bs, nb, T, dh, offs, n_seq, o, st)) != cudaSuccess) break;
         // h = y~ + o Wo^T, in place over y~
         e = launch_gemm_simt(o, true, dh, Wo, true, dh, DUST_F32, M, d, dh, yt, d, 1, part,
                              gemm_simt_splits(M, d, dh), st);

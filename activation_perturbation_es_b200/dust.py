@@ -82,6 +82,9 @@ _SIGS = {
     "dust_toy_suffix_losses": ([_vp, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp, _Noise, _vp, _vp,
                                 _vp, _sz, _vp], _i),
     "dust_toy_suffix_workspace": ([_i, _i, _i, _i, _i], _sz),
+    "dust_attention_internal_costs": ([_vp, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _vp, _Noise, _vp, _vp, _sz,
+                                       _vp], _i),
+    "dust_attention_internal_costs_workspace": ([_i, _i, _i, _i], _sz),
 }
 
 
@@ -367,3 +370,19 @@ def toy_suffix_losses(Y, seq_offsets, Wq, Wk, Wv, Wo, Wout, targets, noise: Nois
                                         _dev(targets, "targets", torch.int32), noise.c(), loss.data_ptr(),
                                         c.data_ptr(), ws.data_ptr(), ws.numel(), _stream()))
     return loss, c
+
+
+def attention_internal_costs(Y, seq_offsets, Wq, Wk, Wv, Wo, which: int, G, noise: Noise):
+    """Costs of the draws of projection `which` (0 q, 1 k, 2 v) scored through the
+    attention output against its estimated error G: c [draw_count][T]."""
+    T, d = Y.shape
+    dh = Wq.shape[0]
+    c = torch.empty(noise.draw_count, T, dtype=torch.float32, device=Y.device)
+    ws = workspace(lib().dust_attention_internal_costs_workspace(noise.draw_count, T, d, dh), Y.device)
+    f32 = torch.float32
+    _check(lib().dust_attention_internal_costs(_dev(Y, "Y", f32), T, d, _dev(seq_offsets, "seq_offsets", torch.int32),
+                                               seq_offsets.numel() - 1, _dev(Wq, "Wq", f32), _dev(Wk, "Wk", f32),
+                                               _dev(Wv, "Wv", f32), _dev(Wo, "Wo", f32), dh, int(which),
+                                               _dev(G, "G", f32), noise.c(), c.data_ptr(), ws.data_ptr(), ws.numel(),
+                                               _stream()))
+    return c

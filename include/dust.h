@@ -271,6 +271,26 @@ dust_status dust_toy_suffix_losses(const float *Y, int T, int d, const int32_t *
                                    void *ws, size_t ws_bytes, void *stream);
 size_t dust_toy_suffix_workspace(int draw_count, int T, int d, int dh, int V);
 
+/* Attention-internal scoring (cnblogs Dust explainer, section
+ * "真正的工作量：压住干扰", second measure): the draws of one internal
+ * projection of a causal softmax attention head (which: 0 = q, 1 = k,
+ * 2 = v; noise channel = projection channel, dh wide) are scored through the
+ * attention output z = Attn(q, k, v) Wo^T against its estimated error G:
+ *   c[k][t] = -< z~_t - z_t, G_t >   (first order: the loss change l~ - l),
+ * computed as -< o~_t - o_t, G_t Wo > since z is linear in the attention's
+ * value output o.  q, k, v = Y Wq^T, Y Wk^T, Y Wv^T (scores / sqrt(dh)),
+ * one head per sequence.  Y, G: [T][d]; Wq, Wk, Wv: [dh][d]; Wo: [d][dh];
+ * c: [draw_count][T].  The costs feed dust_layer_estimate with d_out = dh
+ * (the pages give keys and values a discount gamma close to 1).
+ * Supported: dh % 4 == 0, dh <= 128.  fp32 CUDA cores.
+ * Workspace: dust_attention_internal_costs_workspace(). */
+dust_status dust_attention_internal_costs(const float *Y, int T, int d, const int32_t *seq_offsets,
+                                          int n_seq, const float *Wq, const float *Wk,
+                                          const float *Wv, const float *Wo, int dh, int which,
+                                          const float *G, dust_noise nz, float *c, void *ws,
+                                          size_t ws_bytes, void *stream);
+size_t dust_attention_internal_costs_workspace(int draw_count, int T, int d, int dh);
+
 #ifdef __cplusplus
 }
 #endif

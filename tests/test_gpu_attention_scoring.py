@@ -1,0 +1,85 @@
+"""Attention-internal scoring on the GPU against the oracle, and the estimate
+built on it (reward scan with gamma = 1, draw reduction over the dh
+projection channels, weight estimate against the projection's input)."""
+import numpy as np
+import pytest
+import torch
+
+from activation_perturbation_es_b200 import dust
+from activation_perturbation_es_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    dust.lib()
+
+
+def rel_err(gpu, orc):
+    return float(np.max(np.abs(np.asarray(gpu, np.float64) - orc)) / np.max(np.abs(orc)))
+
+
+def cu(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _block(T=1024, n_seq=4, d=256, dh=64, seed=50):
+    r = np.random.Generator(np.random.PCG64(seed))
+    f = lambda *s, sc=1.0: (r.standard_normal(s) * sc).astype(np.float32)
+    return dict(Y=f(T, d), Wq=f(dh, d, sc=d ** -0.5), Wk=f(dh, d, sc=d ** -0.5), Wv=f(dh, d, sc=d ** -0.5),
+                Wo=f(d, dh, sc=dh ** -0.5), G=f(T, d, sc=0.1), off=I.uniform_offsets(n_seq, T // n_seq))
+
+
+@pytest.mark.parametrize("which", [0, 1, 2])
+def test_attention_costs_parity(orc, which):
+    p = _block()
+    nz = dust.Noise(3, 20 + which, 7, 5, 5, 0.01)
+    c = dust.attention_internal_costs(cu(p["Y"]), cu(p["off"]), cu(p["Wq"]), cu(p["Wk"]), cu(p["Wv"]), cu(p["Wo"]),
+                                      which, cu(p["G"]), nz).cpu().numpy()
+    ref = orc.attention_internal_costs(p["Y"], p["off"], p["Wq"], p["Wk"], p["Wv"], p["Wo"], which, p["G"], 3,
+                                       20 + which, 0.01, np.arange(7, 12))
+    # c is a difference of attention outputs (perturbed minus clean) in fp32
+    assert rel_err(c, ref) < 1e-3
+
+
+def test_value_projection_estimate_end_to_end(orc):
+    p = _block(seed=51)
+    K, dh = 48, 64
+    nz = dust.Noise(4, 22, 0, K, K, 0.01)
+    goff = cu(p["off"])
+    c = dust.attention_internal_costs(cu(p["Y"]), goff, cu(p["Wq"]), cu(p["Wk"]), cu(p["Wv"]), cu(p["Wo"]), 2,
+                                      cu(p["G"]), nz)
+    g, _ = dust.layer_estimate(c, False, goff, 1.0, nz, dh)
+    G_W = dust.weight_grad(g, cu(p["Y"]))                  # the value projection's input is Y
+    toks = np.array([0, 255, 256, 1023])
+    c_h = c.cpu().numpy()
+    g_ref = orc.layer_estimate(c_h, False, dh, p["off"], 1.0, 4, 22, 0, K, 0.01, toks)
+    assert rel_err(g.cpu().numpy()[toks], g_ref) < 1e-3
+    rows = np.array([0, 63])
+    assert rel_err(G_W.cpu().numpy()[rows], orc.weight_grad(g.cpu().numpy(), p["Y"], rows=rows)) < 1e-5
+
+
+def test_value_estimate_converges_through_uniform_attention():
+    """Wq = Wk = 0: E[g_hat_t] = sum_{s >= t} (G_s Wo) / n_s (backprop of <z, G> to v_t)."""
+    T, d, dh, K, sigma = 64, 16, 16, 65536, 0.05
+    p = _block(T=T, n_seq=2, d=d, dh=dh, seed=52)
+    p["Wq"][:] = 0
+    p["Wk"][:] = 0
+    off = p["off"]
+    w = p["G"].astype(np.float64) @ p["Wo"].astype(np.float64)
+    target = np.zeros((T, dh))
+    for q in range(2):
+        for t in range(off[q], off[q + 1]):
+            for s in range(t, off[q + 1]):
+                target[t] += w[s] / (s - off[q] + 1)
+    nz = dust.Noise(5, 23, 0, K, K, sigma)
+    goff = cu(off)
+    c = dust.attention_internal_costs(cu(p["Y"]), goff, cu(p["Wq"]), cu(p["Wk"]), cu(p["Wv"]), cu(p["Wo"]), 2,
+                                      cu(p["G"]), nz)
+    g, _ = dust.layer_estimate(c, False, goff, 1.0, nz, dh)
+    g = g.cpu().numpy().astype(np.float64)
+    cos = np.sum(g * target) / (np.linalg.norm(g) * np.linalg.norm(target))
+    assert cos > 0.98, cos
