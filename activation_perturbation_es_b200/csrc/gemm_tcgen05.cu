@@ -34,7 +34,6 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBK = 64;          // bf16 elements = 128 bytes = one swizzle row
 constexpr int kStages = 4;
-constexpr int kThreads = 128;
 constexpr uint32_t kWaitLimit = 1u << 22;   // polls of a single mbarrier (with back-off: seconds)
 
 // ------------------------------------------------------------------ PTX wrappers
@@ -153,159 +152,225 @@ struct Smem {
     static constexpr int kABytes = kBM * kBK * 2;   // 16 KB
     static constexpr int kBBytes = BN * kBK * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+    static constexpr int kEpiBytes = 8 * 32 * 32 * 4;   // per epilogue warp: a 32 x 32 fp32 tile (xor-swizzled)
+    static constexpr int kBytes = kStages * kStageBytes + kEpiBytes + 1024 /*align*/ + 256 /*barriers*/;
 };
 
-// A: K-major (rows m, 128-byte K rows) or MN-major (two 64-wide MN atoms of
-// 64 K rows each).  Same for B with BN rows / BN/64 atoms.
+// Bounded wait that also gives up as soon as another role has aborted.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag) {
+    for (uint32_t it = 0; it < kWaitLimit; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (it > 64) __nanosleep(256);
+    }
+    return false;
+}
+
+struct Unit {       // one output tile and k slice
+    int m0, n0, kb, nk;
+};
+
+__device__ __forceinline__ Unit unit_of(int u, int tiles_m, int tiles_n, int BN, int K, int k_per_split) {
+    Unit w;
+    const int n_t = u % tiles_n;
+    const int rest = u / tiles_n;
+    const int m_t = rest % tiles_m;
+    const int split = rest / tiles_m;
+    w.m0 = m_t * kBM;
+    w.n0 = n_t * BN;
+    w.kb = split * k_per_split;
+    const int ke = min(K, w.kb + k_per_split);
+    w.nk = ke > w.kb ? (ke - w.kb + kBK - 1) / kBK : 0;
+    return w;
+}
+
+constexpr int kEpiWarps = 8;                          // two per TMEM lane quarter
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;     // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+
+// Persistent, warp-specialised: every CTA walks the work units (tile, k
+// slice) u = blockIdx.x, blockIdx.x + gridDim.x, ...  Two TMEM accumulators
+// of BN columns let the epilogue of one unit overlap the mainloop of the
+// next.  A: K-major (rows m, 128-byte K rows) or MN-major (two 64-wide MN
+// atoms of 64 K rows each); B likewise with BN rows / BN/64 atoms.
 template <int BN, bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, int M, int N,
-               int K, int k_per_split, float* __restrict__ C, int ldc, int accumulate, float* __restrict__ partial,
-               uint32_t* __restrict__ status) {
+               int K, int k_per_split, int splits, float* __restrict__ C, int ldc, int accumulate,
+               float* __restrict__ partial, uint32_t* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     using S = Smem<BN>;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * S::kStageBytes);
+    float* epi = reinterpret_cast<float*>(smem + kStages * S::kStageBytes);   // [8 warps][32][32]
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * S::kStageBytes + S::kEpiBytes);
     uint64_t* empty = full + kStages;
-    uint64_t* done = empty + kStages;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    uint64_t* tfull = empty + kStages;       // [2] accumulator ready for the epilogue
+    uint64_t* tempty = tfull + 2;            // [2] accumulator drained by the epilogue
+    uint64_t* drain = tempty + 2;            // MMAs in flight at an abort
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM;
-    const int kb = blockIdx.z * k_per_split;
-    const int ke = min(K, kb + k_per_split);
-    const int nk = ke > kb ? (ke - kb + kBK - 1) / kBK : 0;
+    const int tiles_m = (M + kBM - 1) / kBM, tiles_n = (N + BN - 1) / BN;
+    const int units = tiles_m * tiles_n * splits;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(done, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], kEpiWarps);
+        }
+        mbar_init(drain, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 1) tmem_alloc(tmem_slot, BN);
+    if (warp == 1) tmem_alloc(tmem_slot, 2 * BN);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    bool ok = true;
-    if (warp == 0 && lane == 0 && nk > 0) {
-        // ---------------- TMA producer
-        int issued = 0;
-        for (int it = 0; it < nk && ok; ++it) {
-            const int s = it % kStages;
-            if (it >= kStages && !mbar_wait(&empty[s], ((it / kStages) - 1) & 1)) { ok = false; break; }
-            if (*abort_flag) { ok = false; break; }
-            uint8_t* sa = smem + s * S::kStageBytes;
-            uint8_t* sb = sa + S::kABytes;
-            mbar_arrive_expect_tx(&full[s], S::kStageBytes);
-            const int k0 = kb + it * kBK;
-            if (A_MN) {
-                tma_load_2d(sa, &map_a, &full[s], m0, k0);
-                tma_load_2d(sa + 64 * kBK * 2, &map_a, &full[s], m0 + 64, k0);
-            } else {
-                tma_load_2d(sa, &map_a, &full[s], k0, m0);
-            }
-            if (B_MN) {
-#pragma unroll
-                for (int h = 0; h < BN / 64; ++h) tma_load_2d(sb + h * 64 * kBK * 2, &map_b, &full[s], n0 + 64 * h, k0);
-            } else {
-                tma_load_2d(sb, &map_b, &full[s], k0, n0);
-            }
-            issued = it + 1;
-        }
-        if (!ok) {
-            atomicExch(status, kStatusTimeout);
-            *abort_flag = 1;
-        }
-        // drain: the last (up to kStages) loads must land before the CTA exits
-        for (int it = issued > kStages ? issued - kStages : 0; it < issued; ++it)
-            mbar_wait(&full[it % kStages], (it / kStages) & 1);
-    } else if (warp == 1 && lane == 0 && nk > 0) {
-        // ---------------- MMA issuer
-        constexpr uint32_t idesc = instr_desc(BN, A_MN, B_MN);
-        for (int it = 0; it < nk; ++it) {
-            const int s = it % kStages;
-            if (!mbar_wait(&full[s], (it / kStages) & 1) || *abort_flag) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t sa = smem_u32(smem + s * S::kStageBytes);
-            const uint32_t sb = sa + S::kABytes;
-#pragma unroll
-            for (int j = 0; j < kBK / 16; ++j) {
-                // K-major: the 16-element k step is 32 bytes along the swizzled row;
-                // MN-major: it is 16 rows of 128 bytes.
-                const uint64_t ad = A_MN ? smem_desc(sa + j * 16 * 128, 64 * kBK * 2, 1024)
-                                         : smem_desc(sa + j * 32, 16, 1024);
-                const uint64_t bd = B_MN ? smem_desc(sb + j * 16 * 128, 64 * kBK * 2, 1024)
-                                         : smem_desc(sb + j * 32, 16, 1024);
-                tc_mma(tmem, ad, bd, idesc, (it > 0 || j > 0) ? 1u : 0u);
-            }
-            tc_commit(&empty[s]);
-        }
-        if (!ok) {
-            atomicExch(status, kStatusTimeout);
-            *abort_flag = 1;
-        }
-        tc_commit(done);   // arrives once every MMA issued above has completed
-    }
-    __syncwarp();
-
-    // ---------------- epilogue: TMEM -> registers -> global
-    bool have = nk > 0;
-    if (have) {
-        if (!mbar_wait(done, 0)) {
-            if (lane == 0) atomicExch(status, kStatusTimeout);
-            have = false;
-        }
-    }
-    have = have && !*abort_flag;
-    have = __all_sync(0xffffffffu, have);   // tcgen05.ld is warp-collective
-    tc_fence_after();
-    const int row = m0 + warp * 32 + lane;
-#pragma unroll 1
-    for (int c0 = 0; c0 < BN; c0 += 32) {
-        float v[32];
-        if (have) {
-            tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(c0), v);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-        }
-        if (row >= M) continue;
-        const int col = n0 + c0;
-        if (partial != nullptr) {
-            float* dst = partial + (static_cast<size_t>(blockIdx.z) * M + row) * N + col;
-            if (col + 32 <= N && (N & 3) == 0) {
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-            } else {
-                for (int i = 0; i < 32 && col + i < N; ++i) dst[i] = v[i];
-            }
-        } else {
-            float* dst = C + static_cast<size_t>(row) * ldc + col;
-            if (col + 32 <= N && (ldc & 3) == 0) {
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    float4 o = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-                    if (accumulate) {
-                        const float4 p = *reinterpret_cast<float4*>(dst + i);
-                        o.x += p.x; o.y += p.y; o.z += p.z; o.w += p.w;
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer
+            int it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                const Unit w = unit_of(u, tiles_m, tiles_n, BN, K, k_per_split);
+                for (int kk = 0; kk < w.nk; ++kk, ++it) {
+                    const int s = it % kStages;
+                    if (it >= kStages && !mbar_wait_or_abort(&empty[s], ((it / kStages) - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
                     }
-                    *reinterpret_cast<float4*>(dst + i) = o;
+                    uint8_t* sa = smem + s * S::kStageBytes;
+                    uint8_t* sb = sa + S::kABytes;
+                    mbar_arrive_expect_tx(&full[s], S::kStageBytes);
+                    const int k0 = w.kb + kk * kBK;
+                    if (A_MN) {
+                        tma_load_2d(sa, &map_a, &full[s], w.m0, k0);
+                        tma_load_2d(sa + 64 * kBK * 2, &map_a, &full[s], w.m0 + 64, k0);
+                    } else {
+                        tma_load_2d(sa, &map_a, &full[s], k0, w.m0);
+                    }
+                    if (B_MN) {
+#pragma unroll
+                        for (int h = 0; h < BN / 64; ++h)
+                            tma_load_2d(sb + h * 64 * kBK * 2, &map_b, &full[s], w.n0 + 64 * h, k0);
+                    } else {
+                        tma_load_2d(sb, &map_b, &full[s], k0, w.n0);
+                    }
                 }
-            } else {
-                for (int i = 0; i < 32 && col + i < N; ++i) dst[i] = accumulate ? dst[i] + v[i] : v[i];
             }
+            if (!ok) {
+                atomicExch(status, kStatusTimeout);
+                *abort_flag = 1;
+            }
+            // the last (up to kStages) loads must land before the CTA exits
+            for (int j = it > kStages ? it - kStages : 0; j < it; ++j) mbar_wait(&full[j % kStages], (j / kStages) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer
+            constexpr uint32_t idesc = instr_desc(BN, A_MN, B_MN);
+            int it = 0, tcount = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++tcount) {
+                const Unit w = unit_of(u, tiles_m, tiles_n, BN, K, k_per_split);
+                const int buf = tcount & 1;
+                if (tcount >= 2 && !mbar_wait_or_abort(&tempty[buf], ((tcount >> 1) - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t acc = tmem + static_cast<uint32_t>(buf * BN);
+                for (int kk = 0; kk < w.nk; ++kk, ++it) {
+                    const int s = it % kStages;
+                    if (!mbar_wait_or_abort(&full[s], (it / kStages) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + s * S::kStageBytes);
+                    const uint32_t sb = sa + S::kABytes;
+#pragma unroll
+                    for (int j = 0; j < kBK / 16; ++j) {
+                        // K-major: a 16-element k step is 32 bytes along the swizzled row;
+                        // MN-major: it is 16 rows of 128 bytes.
+                        const uint64_t ad = A_MN ? smem_desc(sa + j * 16 * 128, 64 * kBK * 2, 1024)
+                                                 : smem_desc(sa + j * 32, 16, 1024);
+                        const uint64_t bd = B_MN ? smem_desc(sb + j * 16 * 128, 64 * kBK * 2, 1024)
+                                                 : smem_desc(sb + j * 32, 16, 1024);
+                        tc_mma(acc, ad, bd, idesc, (kk > 0 || j > 0) ? 1u : 0u);
+                    }
+                    tc_commit(&empty[s]);
+                }
+                if (!ok) break;
+                tc_commit(&tfull[buf]);   // arrives once this unit's MMAs have completed
+            }
+            if (!ok) {
+                atomicExch(status, kStatusTimeout);
+                *abort_flag = 1;
+            }
+            tc_commit(drain);             // every MMA issued above has completed when this arrives
+            mbar_wait(drain, 0);
+        }
+    } else {
+        // ---------------- epilogue: TMEM -> registers -> global (warps 2-9)
+        const int quarter = warp & 3;     // the TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2; // the two warps of a quarter take alternate 32-column blocks
+        int tcount = 0;
+        for (int u = blockIdx.x; u < units; u += gridDim.x, ++tcount) {
+            const Unit w = unit_of(u, tiles_m, tiles_n, BN, K, k_per_split);
+            const int buf = tcount & 1;
+            bool have = mbar_wait_or_abort(&tfull[buf], (tcount >> 1) & 1, abort_flag);
+            if (!__all_sync(0xffffffffu, have)) break;
+            tc_fence_after();
+            have = w.nk > 0;
+            const int split = u / (tiles_m * tiles_n);
+            // Each 32 x 32 block (this warp's 32 rows x 32 columns) goes through a
+            // padded shared tile so that the global stores are row segments:
+            // after the transpose lane l holds column c0 + l of every row.
+            float* tile = epi + (warp - 2) * (32 * 32);
+            const int row0 = w.m0 + quarter * 32;
+            float* base = partial != nullptr ? partial + static_cast<size_t>(split) * M * N : C;
+            const int ld = partial != nullptr ? N : ldc;
+            const bool add = partial == nullptr && accumulate;
+#pragma unroll 1
+            for (int c0 = 32 * half; c0 < BN; c0 += 64) {
+                float v[32];
+                if (have) {
+                    tmem_ld32(tmem + static_cast<uint32_t>(buf * BN + c0) + (static_cast<uint32_t>(quarter * 32) << 16), v);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) tile[lane * 32 + (i ^ lane)] = v[i];
+                __syncwarp();
+                const int col = w.n0 + c0 + lane;
+                if (col < N) {
+#pragma unroll 4
+                    for (int r = 0; r < 32; ++r) {
+                        const int row = row0 + r;
+                        if (row >= M) break;
+                        float* dst = base + static_cast<size_t>(row) * ld + col;
+                        const float x = tile[r * 32 + (lane ^ r)];
+                        *dst = add ? *dst + x : x;
+                    }
+                }
+                __syncwarp();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&tempty[buf])) : "memory");
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) tmem_dealloc(tmem, BN);
+    if (warp == 1) tmem_dealloc(tmem, 2 * BN);
 }
 
 // One thread waits, with the pipeline's bounded-wait code, on an mbarrier that
@@ -352,6 +417,18 @@ bool make_map(CUtensorMap* map, const void* base, int inner, int outer, int ld, 
 
 int pick_bn(int N) { return N >= 256 ? 256 : (N > 64 ? 128 : 64); }
 
+int sm_count() {
+    static int n = 0;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = kNumSMs;
+    });
+    return n;
+}
+
 template <int BN, bool A_MN, bool B_MN>
 cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int K, int kps, int splits,
                      float* C, int ldc, int accumulate, float* partial, uint32_t* status, cudaStream_t st) {
@@ -362,10 +439,11 @@ cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N,
         attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<BN>::kBytes);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    const dim3 grid(static_cast<unsigned>(ceil_div(N, BN)), static_cast<unsigned>(ceil_div(M, kBM)),
-                    static_cast<unsigned>(splits));
-    kern<<<grid, kThreads, Smem<BN>::kBytes, st>>>(ma, mb, M, N, K, kps, C, ldc, accumulate,
-                                                    splits > 1 ? partial : nullptr, status);
+    const long long units = ceil_div(N, BN) * ceil_div(M, kBM) * splits;
+    const int per_sm = Smem<BN>::kBytes * 2 <= 227 * 1024 ? 2 : 1;   // TMEM: 2 x 2 BN <= 512 columns for BN <= 128
+    const long long grid = units < static_cast<long long>(sm_count()) * per_sm ? units : sm_count() * per_sm;
+    kern<<<static_cast<unsigned>(grid), kGemmThreads, Smem<BN>::kBytes, st>>>(
+        ma, mb, M, N, K, kps, splits, C, ldc, accumulate, splits > 1 ? partial : nullptr, status);
     return cudaGetLastError();
 }
 
@@ -396,12 +474,24 @@ bool gemm_tc_supported(int M, int N, int K, bool a_kmajor, bool b_kmajor) {
 }
 
 int gemm_tc_splits(int M, int N, int K) {
+    // Work units are (tile, k slice); the persistent grid (one CTA per SM)
+    // walks them in rounds.  Pick the split of k that keeps the most SMs busy
+    // over all rounds, keeping slices of at least 16 k blocks; on a tie the
+    // smaller split wins (partial tiles cost HBM traffic and a reduction).
     const long long tiles = ceil_div(M, kBM) * ceil_div(N, pick_bn(N));
     const long long kblocks = ceil_div(K, kBK);
-    // enough CTAs for several waves over the SMs, slices of at least 8 k blocks
-    long long s = 1;
-    while (tiles * s < 4LL * kNumSMs && kblocks / (s * 2) >= 8 && s < 32) s *= 2;
-    return static_cast<int>(s);
+    const long long grid = kNumSMs;
+    long long best_s = 1;
+    double best_u = 0.0;
+    for (long long s = 1; s <= 32 && (s == 1 || kblocks / s >= 16); s *= 2) {
+        const long long units = tiles * s;
+        const double util = static_cast<double>(units) / static_cast<double>(ceil_div(units, grid) * grid);
+        if (util > best_u + 1e-3) {
+            best_u = util;
+            best_s = s;
+        }
+    }
+    return static_cast<int>(best_s);
 }
 
 cudaError_t launch_gemm_tc(const void* A, bool a_kmajor, int lda, const void* B, bool b_kmajor, int ldb, int M, int N,
