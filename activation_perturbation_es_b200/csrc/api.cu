@@ -195,6 +195,8 @@ dust_status dust_reward_scan_split(const float* c, float* r, int K, int T, const
     DUST_TRY(check_ptr(c, "c"));
     DUST_TRY(check_ptr(r, "r"));
     DUST_TRY(check_seq(seq_offsets, n_seq, K, T));
+    DUST_REQUIRE(static_cast<long long>(K) * dust::ceil_div(T, 1024) < (1ll << 31), DUST_ERR_INVALID_ARG,
+                 "draws x token chunks must be < 2^31");
     DUST_TRY(check_ptr(ws, "ws"));
     const size_t need = dust_reward_scan_split_workspace(K, T);
     DUST_REQUIRE(ws_bytes >= need, DUST_ERR_WORKSPACE, "workspace %zu bytes < %zu", ws_bytes, need);
@@ -477,6 +479,7 @@ dust_status dust_synth_costs(const float* u, int T, int d_out, dust_noise nz, fl
     DUST_REQUIRE(std::isfinite(nz.sigma) && nz.sigma >= 0.0f, DUST_ERR_INVALID_ARG, "sigma must be finite and >= 0");
     DUST_REQUIRE(std::isfinite(eps_scale), DUST_ERR_INVALID_ARG, "eps_scale must be finite");
     DUST_REQUIRE(T > 0 && d_out > 0, DUST_ERR_INVALID_ARG, "T and d_out must be > 0");
+    DUST_REQUIRE(nz.draw_count <= 65535u * 32u, DUST_ERR_INVALID_ARG, "draw_count must be <= 2097120");
     DUST_TRY(check_ptr(u, "u"));
     DUST_TRY(check_ptr(c, "c"));
     return cuda_status(dust::launch_synth_costs(u, T, d_out, nz, eps_scale, c, as_stream(stream)), "dust_synth_costs");

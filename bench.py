@@ -328,7 +328,7 @@ def main():
     e2e = None if args.no_e2e else e2e_run(step, args, world)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, K, budget_s=20.0)
+        cpu = cpu_baseline(w, K)
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -526,7 +526,7 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(w, K, budget_s=20.0):
+def cpu_baseline(w, K):
     cores = cpu_cores()
     n_tok = max(2, min(512, 2 * cores))
     t_s, units, t_full = oracle_sample(w, K, n_tok)
