@@ -353,8 +353,8 @@ dust_status dust_head_step(const void* X, const void* W, dust_dtype dt, const fl
     DUST_REQUIRE(dt == DUST_F32 || dt == DUST_BF16, DUST_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
     DUST_REQUIRE(T > 0 && V > 0, DUST_ERR_INVALID_ARG, "T and V must be > 0");
     DUST_REQUIRE(Vc > 0 && V % Vc == 0, DUST_ERR_INVALID_ARG, "Vc=%d must divide V=%d", Vc, V);
-    DUST_REQUIRE(Vc % 128 == 0 && Vc <= 1024, DUST_ERR_UNSUPPORTED,
-                 "Vc=%d unsupported (a multiple of 128, at most 1024)", Vc);
+    DUST_REQUIRE(dust::head_chunk_supported(Vc), DUST_ERR_UNSUPPORTED,
+                 "Vc=%d unsupported (multiples of 128 up to 1024, of 256 up to 2048, of 512 up to 4096)", Vc);
     DUST_REQUIRE(V / Vc <= 65535, DUST_ERR_INVALID_ARG, "too many chunks");
     const bool has_Z = Z != nullptr, want_G_W = G_W != nullptr;
     if (!has_Z || want_G_W) {

@@ -83,20 +83,29 @@ __device__ __forceinline__ float expm1_series(float x) {
 
 constexpr int kHeadWarps = 4;   // tokens per block
 
-template <int QPL, int TIER>   // channel quads per lane: Vc = 128 * QPL; expm1 tier (see expm1_series)
+// WPT warps share one token's chunk when it is wider than 1024 vocab ids (the
+// "whole vocabulary" reading Vc = V of the LM-head pass): each warp covers
+// 128 * QPL ids; per draw the warps' partial sums meet in shared memory
+// (double-buffered by draw parity, one named barrier per draw) and every warp
+// adds them in the same fixed order, so all get the same c.
+template <int QPL, int TIER, int WPT>
 __global__ void __launch_bounds__(32 * kHeadWarps)
 head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
                   const int32_t* __restrict__ targets, int T, int V, int Vc, uint32_t seed, uint32_t layer,
                   uint32_t draw_begin, int nd, float sigma, float scale, float* __restrict__ c_out,
                   float* __restrict__ g, __nv_bfloat16* __restrict__ g16, int accumulate) {
-    // the chunk's softmax probabilities of each warp's token: read every draw,
-    // so they live in shared memory and leave the registers to a and g
+    constexpr int kTPB = kHeadWarps / WPT;        // tokens per block
+    constexpr int kSub = 128 * QPL;               // vocab ids per warp
+    // the softmax probabilities of each warp's ids: read every draw, so they
+    // live in shared memory and leave the registers to a and g
     __shared__ float4 p_s[kHeadWarps][32 * QPL];
+    __shared__ float red_s[kTPB][2][WPT], red_ay[kTPB][2][WPT];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * kHeadWarps + warp;
-    if (t >= T) return;
+    const int ts = warp / WPT, part = warp % WPT;
+    const int t = blockIdx.x * kTPB + ts;
+    if (t >= T) return;                           // the token's warps leave together
     const int chunk = blockIdx.y;
-    const int v0 = chunk * Vc;
+    const int v0 = chunk * Vc + part * kSub;      // first id of this warp
     const float* zt = Z + static_cast<size_t>(t) * V;
     const float l = __ldg(lse + t);
     float4* p = p_s[warp];
@@ -106,12 +115,14 @@ head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
         p[lane + 32 * k] = make_float4(expf(z.x - l), expf(z.y - l), expf(z.z - l), expf(z.w - l));
     }
     __syncwarp();
-    const int rel = clamp_int(__ldg(targets + t), 0, V - 1) - v0;
-    const bool in_chunk = rel >= 0 && rel < Vc;
-    const int owner = in_chunk ? ((rel >> 2) & 31) : 0;
-    const int ky = in_chunk ? (rel >> 7) : -1;
+    const int rel_chunk = clamp_int(__ldg(targets + t), 0, V - 1) - chunk * Vc;
+    const bool in_chunk = rel_chunk >= 0 && rel_chunk < Vc;
+    const int rel = rel_chunk - part * kSub;
+    const bool in_mine = rel >= 0 && rel < kSub;
+    const int owner = in_mine ? ((rel >> 2) & 31) : 0;
+    const int ky = in_mine ? (rel >> 7) : -1;
     const int wy = rel & 3;
-    const bool i_own = in_chunk && lane == owner;
+    const bool i_own = in_mine && lane == owner;
 
     float gacc[QPL][4];
 #pragma unroll
@@ -136,9 +147,25 @@ head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
             if (i_own && k == ky) ay = wy == 0 ? n.x : (wy == 1 ? n.y : (wy == 2 ? n.z : n.w));
         }
         S = warp_sum(S);
-        ay = __shfl_sync(0xffffffffu, ay, owner);
-        const float c = log1pf(S) - (in_chunk ? sigma * ay : 0.0f);
-        if (c_out != nullptr && lane == 0) c_out[(static_cast<size_t>(chunk) * nd + i) * T + t] = c;
+        ay = __shfl_sync(0xffffffffu, ay, owner);      // 0 unless this warp holds the target
+        float sy = in_mine ? sigma * ay : 0.0f;
+        if (WPT > 1) {
+            const int par = i & 1;
+            if (lane == 0) {
+                red_s[ts][par][part] = S;
+                red_ay[ts][par][part] = sy;
+            }
+            asm volatile("bar.sync %0, %1;" ::"r"(1 + ts), "r"(32 * WPT) : "memory");
+            S = 0.0f;
+            sy = 0.0f;
+#pragma unroll
+            for (int w = 0; w < WPT; ++w) {
+                S += red_s[ts][par][w];
+                sy += red_ay[ts][par][w];
+            }
+        }
+        const float c = log1pf(S) - (in_chunk ? sy : 0.0f);
+        if (c_out != nullptr && lane == 0 && part == 0) c_out[(static_cast<size_t>(chunk) * nd + i) * T + t] = c;
 #pragma unroll
         for (int k = 0; k < QPL; ++k)
 #pragma unroll
@@ -174,39 +201,72 @@ cudaError_t launch_row_stats(const float* Z, const int32_t* targets, int T, int 
     return cudaGetLastError();
 }
 
+// Supported chunk widths: a multiple of 128 up to 1024 (one warp per token),
+// of 256 up to 2048 (two warps) or of 512 up to 4096 (four warps).
+bool head_chunk_supported(int Vc) {
+    return (Vc > 0 && Vc <= 1024 && Vc % 128 == 0) || (Vc > 1024 && Vc <= 2048 && Vc % 256 == 0) ||
+           (Vc > 2048 && Vc <= 4096 && Vc % 512 == 0);
+}
+
+namespace {
+
+template <int QPL, int WPT>
+void launch_qw(int tier, dim3 grid, cudaStream_t st, const float* Z, const float* lse, const int32_t* targets, int T,
+               int V, int Vc, const dust_noise& nz, float scale, float* c_out, float* g, __nv_bfloat16* g16,
+               int accumulate) {
+    const int nd = static_cast<int>(nz.draw_count);
+#define DUST_HEAD_TIER(TIER_)                                                                               \
+    head_chunk_kernel<QPL, TIER_, WPT><<<grid, 32 * kHeadWarps, 0, st>>>(Z, lse, targets, T, V, Vc, nz.seed,  \
+                                                                         nz.layer, nz.draw_begin, nd, nz.sigma, \
+                                                                         scale, c_out, g, g16, accumulate)
+    if (tier == 2) DUST_HEAD_TIER(2);
+    else if (tier == 1) DUST_HEAD_TIER(1);
+    else DUST_HEAD_TIER(0);
+#undef DUST_HEAD_TIER
+}
+
+}  // namespace
+
 cudaError_t launch_head_chunks(const float* Z, const float* lse, const int32_t* targets, int T, int V, int Vc,
                                const dust_noise& nz, float* c_out, float* g, void* g_bf16, int accumulate,
                                cudaStream_t stream) {
-    const dim3 grid(static_cast<unsigned>(ceil_div(T, kHeadWarps)), static_cast<unsigned>(V / Vc));
+    if (!head_chunk_supported(Vc)) return cudaErrorNotSupported;
+    const int wpt = Vc <= 1024 ? 1 : (Vc <= 2048 ? 2 : 4);
+    const int qpl = Vc / (128 * wpt);
+    const dim3 grid(static_cast<unsigned>(ceil_div(T, kHeadWarps / wpt)), static_cast<unsigned>(V / Vc));
     // |a| < 5.66 for every draw the generator produces (see expm1_series)
     const int tier = nz.sigma <= 0.01f ? 2 : (nz.sigma <= 0.02f ? 1 : 0);
     const float scale = static_cast<float>(-1.0 / (static_cast<double>(nz.K_total) * nz.sigma));
     auto* g16 = static_cast<__nv_bfloat16*>(g_bf16);
-    const int nd = static_cast<int>(nz.draw_count);
-#define DUST_HEAD_TIER(Q, TIER_)                                                                           \
-    head_chunk_kernel<Q, TIER_><<<grid, 32 * kHeadWarps, 0, stream>>>(Z, lse, targets, T, V, Vc, nz.seed,     \
-                                                                      nz.layer, nz.draw_begin, nd, nz.sigma,  \
-                                                                      scale, c_out, g, g16, accumulate)
-#define DUST_HEAD_LAUNCH(Q)                          \
-    do {                                             \
-        if (tier == 2) DUST_HEAD_TIER(Q, 2);         \
-        else if (tier == 1) DUST_HEAD_TIER(Q, 1);    \
-        else DUST_HEAD_TIER(Q, 0);                   \
-    } while (0)
-    if (Vc % 128 != 0) return cudaErrorNotSupported;
-    switch (Vc / 128) {
-        case 1: DUST_HEAD_LAUNCH(1); break;
-        case 2: DUST_HEAD_LAUNCH(2); break;
-        case 3: DUST_HEAD_LAUNCH(3); break;
-        case 4: DUST_HEAD_LAUNCH(4); break;
-        case 5: DUST_HEAD_LAUNCH(5); break;
-        case 6: DUST_HEAD_LAUNCH(6); break;
-        case 7: DUST_HEAD_LAUNCH(7); break;
-        case 8: DUST_HEAD_LAUNCH(8); break;
-        default: return cudaErrorNotSupported;
+#define DUST_HEAD_QW(Q, W)                                                                            \
+    launch_qw<Q, W>(tier, grid, stream, Z, lse, targets, T, V, Vc, nz, scale, c_out, g, g16, accumulate)
+    if (wpt == 1) {
+        switch (qpl) {
+            case 1: DUST_HEAD_QW(1, 1); break;
+            case 2: DUST_HEAD_QW(2, 1); break;
+            case 3: DUST_HEAD_QW(3, 1); break;
+            case 4: DUST_HEAD_QW(4, 1); break;
+            case 5: DUST_HEAD_QW(5, 1); break;
+            case 6: DUST_HEAD_QW(6, 1); break;
+            case 7: DUST_HEAD_QW(7, 1); break;
+            default: DUST_HEAD_QW(8, 1); break;
+        }
+    } else if (wpt == 2) {
+        switch (qpl) {
+            case 5: DUST_HEAD_QW(5, 2); break;
+            case 6: DUST_HEAD_QW(6, 2); break;
+            case 7: DUST_HEAD_QW(7, 2); break;
+            default: DUST_HEAD_QW(8, 2); break;
+        }
+    } else {
+        switch (qpl) {
+            case 5: DUST_HEAD_QW(5, 4); break;
+            case 6: DUST_HEAD_QW(6, 4); break;
+            case 7: DUST_HEAD_QW(7, 4); break;
+            default: DUST_HEAD_QW(8, 4); break;
+        }
     }
-#undef DUST_HEAD_LAUNCH
-#undef DUST_HEAD_TIER
+#undef DUST_HEAD_QW
     return cudaGetLastError();
 }
 

@@ -61,6 +61,7 @@ bool gemm_tc_supported(int M, int N, int K, bool a_kmajor, bool b_kmajor);
 // a2 row statistics + a3/a5 fused head (head.cu)
 cudaError_t launch_row_stats(const float* Z, const int32_t* targets, int T, int V, float* lse,
                              float* ell, cudaStream_t stream);
+bool head_chunk_supported(int Vc);
 cudaError_t launch_head_chunks(const float* Z, const float* lse, const int32_t* targets, int T,
                                int V, int Vc, const dust_noise& nz, float* c_out, float* g,
                                void* g_bf16, int accumulate, cudaStream_t stream);

@@ -199,7 +199,9 @@ dust_status dust_head_row_stats(const float *Z, const int32_t *targets, int T, i
  *      recomputed into the workspace, a2) and when G_W is requested.
  *   Z: nullable cached logits [T][V] fp32.
  *   targets: [T] int32 in [0, V).
- *   Vc: chunk width; must divide V; supported: a multiple of 128, <= 1024.
+ *   Vc: chunk width; must divide V; supported: multiples of 128 up to 1024,
+ *      of 256 up to 2048 and of 512 up to 4096 (Vc = V is the reading where
+ *      every draw perturbs the whole vocabulary).
  *   c_out: nullable [V/Vc][draw_count][T] fp32, the costs of every pass.
  *   g_hat: [T][V] fp32 (overwritten, or added to when accumulate = 1).
  *   g_hat_bf16: nullable [T][V] bf16 copy of the final g_hat.

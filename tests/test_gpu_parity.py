@@ -268,6 +268,21 @@ def test_head_step_chunks_and_split(orc, sigma):
     assert rel_err(host(part["g_hat"]), host(full["g_hat"])) < 1e-6
 
 
+@pytest.mark.parametrize("V,Vc,sigma", [(2560, 1280, 0.01), (4096, 2048, 0.05), (5120, 2560, 0.01),
+                                         (4096, 4096, 0.02)])
+def test_head_wide_chunks(orc, V, Vc, sigma):
+    """Chunks wider than 1024 ids (2 or 4 warps per token, partial sums met in
+    shared memory), including the whole-vocabulary reading Vc = V."""
+    T, K = 24, 6
+    Z = I.normal((T, V), 1.5, seed=V + Vc)
+    y = I.targets(T, V, seed=V)
+    sub = Vc // (2 if Vc <= 2048 else 4)        # ids per warp
+    y[:6] = [0, sub - 1, sub, Vc - 1, Vc % V, V - 1]   # targets on warp and chunk edges
+    nz = dust.Noise(2, 8, 3, K, K, sigma)
+    out = dust.head_step(cu(y), Vc, nz, Z=cu(Z), want_c=True)
+    _head_check(orc, Z, y, np.arange(T), Vc, nz, out, 1e-4)
+
+
 @pytest.mark.parametrize("K", [64])
 def test_head_pages_sampled(orc, K):
     """HEAD_PAGES at full size (16 x 1024 tokens, V = 4096, Vc = 1024, bf16 X/W),
