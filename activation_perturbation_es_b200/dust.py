@@ -139,12 +139,16 @@ _ws = {}
 
 
 def workspace(nbytes: int, device=None) -> torch.Tensor:
-    """A cached caller-owned workspace of at least nbytes on the current device."""
+    """A cached caller-owned workspace of at least nbytes, one per (device,
+    current stream): calls on one stream run in order and can share it, calls
+    on different streams get different buffers.  Grows (reallocates) on
+    demand, so warm a path up once before capturing it in a CUDA graph."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
-    cur = _ws.get(dev)
+    key = (dev, torch.cuda.current_stream(dev).cuda_stream)
+    cur = _ws.get(key)
     if cur is None or cur.numel() < nbytes:
         cur = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=dev)
-        _ws[dev] = cur
+        _ws[key] = cur
     return cur
 
 
