@@ -400,3 +400,36 @@ def test_attention_value_estimate_converges_to_backprop_through_uniform_attentio
     slope = np.polyfit(np.log(Ks), np.log(errs), 1)[0]
     assert -0.6 <= slope <= -0.4, (slope, errs)
     assert errs[-1] < 0.2, errs
+
+
+def test_suffix_hard_self_attention_limit(orc):
+    """Orthonormal layer outputs y_t, Wq = lam A and Wk = lam A^-T for a
+    non-orthogonal A: the score of token t on u is q_t . k_u / sqrt(dh) =
+    lam^2 <y_t, y_u> / sqrt(dh) = lam^2 delta_tu / sqrt(dh) (while q_t . q_u and
+    k_t . k_u are not), so for large lam every token attends only to itself,
+    o_t = v_t, and the suffix is the residual + readout of y_t + Wo Wv y_t
+    (numpy/scipy closed form).  Together with the uniform case (which pins the
+    causal mask and the value path) this pins the score path q_t . k_u."""
+    d = dh = 8
+    T = 8
+    r = np.random.Generator(np.random.PCG64(60))
+    Q, _ = np.linalg.qr(r.standard_normal((d, d)))
+    X = Q.astype(np.float32)                           # rows orthonormal
+    W = np.eye(d, dtype=np.float32)                    # y = X
+    lam = np.sqrt(300.0 * np.sqrt(dh))                 # self score 300, others 0
+    A = np.linalg.qr(r.standard_normal((d, d)))[0] @ np.diag(np.linspace(0.5, 2.0, d)) @ \
+        np.linalg.qr(r.standard_normal((d, d)))[0].T
+    Wq = (lam * A).astype(np.float32)
+    Wk = (lam * np.linalg.inv(A).T).astype(np.float32)
+    Wv = (r.standard_normal((dh, d)) * 0.5).astype(np.float32)
+    Wo = (r.standard_normal((d, dh)) * 0.5).astype(np.float32)
+    Wout = (r.standard_normal((10, d)) * 0.5).astype(np.float32)
+    y = r.integers(0, 10, T).astype(np.int32)
+    off = np.array([0, 3, T], np.int32)
+    loss = orc.toy_suffix_losses(X, W, off, Wq, Wk, Wv, Wo, Wout, y, 0, 1, 0.0, [0], with_noise=False)[0]
+    Y = X.astype(np.float64)
+    h = Y + Y @ Wv.astype(np.float64).T @ Wo.astype(np.float64).T
+    z = h @ Wout.astype(np.float64).T
+    ref = sp.logsumexp(z, axis=1) - z[np.arange(T), y]
+    # Wq, Wk are rounded to binary32: the off-diagonal scores are ~lam^2 * 1e-7, far from mattering
+    np.testing.assert_allclose(loss, ref, rtol=1e-6)
