@@ -83,8 +83,6 @@ struct Layout {
 
 uint8_t* region(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
 
-size_t dtype_bytes(dust_dtype dt) { return dt == DUST_BF16 ? 2 : 4; }
-
 // ---- GEMM dispatch shared by weight_grad, logits and head_step ----------------
 struct GemmPlan {
     bool tc = false;
