@@ -63,22 +63,33 @@ row_stats_kernel(const float* __restrict__ Z, const int32_t* __restrict__ target
     }
 }
 
-// expm1(x) by its Taylor series, for the small |x| = |sigma a| of the head's
-// perturbations (|a| <= sqrt(46 ln 2) < 5.66 for every a the generator makes):
+// p expm1(sigma a) by the Taylor series of expm1, for the small |x| = |sigma a|
+// of the head's perturbations (|a| <= sqrt(46 ln 2) < 5.66 for every a the
+// generator makes):
 //   tier 1, sigma <= 0.02  (|x| <= 0.114): to x^5, relative truncation < x^5/720 < 3e-8;
 //   tier 2, sigma <= 0.01  (|x| <= 0.057): to x^4, relative truncation < x^4/120 < 9e-8 < 2^-23.
-// Larger sigma (tier 0) uses expm1f.
+// The series is evaluated in a, with sigma's powers in the coefficients
+// (c_k = sigma^k / (k+1)!) and p sigma precomputed:
+//   p expm1(sigma a) = (p sigma) a (1 + a (c_1 + a (c_2 + a (c_3 [+ a c_4])))),
+// one multiply fewer per vocabulary id than forming x = sigma a first.
+// Larger sigma (tier 0) uses expm1f(sigma a) with p itself.
+struct ExpCoef {
+    float c1, c2, c3, c4;
+};
+
+__device__ __forceinline__ ExpCoef exp_coef(float sigma) {
+    return {sigma * 0.5f, sigma * sigma * (1.0f / 6.0f), sigma * sigma * sigma * (1.0f / 24.0f),
+            sigma * sigma * sigma * sigma * (1.0f / 120.0f)};
+}
+
+// S + p expm1(sigma a); pp is p (tier 0) or p sigma (series tiers)
 template <int TIER>
-__device__ __forceinline__ float expm1_series(float x) {
-    float t;
-    if (TIER == 1) {
-        t = fmaf(x, 1.0f / 120.0f, 1.0f / 24.0f);
-        t = fmaf(x, t, 1.0f / 6.0f);
-    } else {
-        t = fmaf(x, 1.0f / 24.0f, 1.0f / 6.0f);
-    }
-    t = fmaf(x, t, 0.5f);
-    return fmaf(x * x, t, x);
+__device__ __forceinline__ float add_p_expm1(float S, float pp, float a, float sigma, const ExpCoef& c) {
+    if (TIER == 0) return fmaf(pp, expm1f(sigma * a), S);
+    float t = TIER == 1 ? fmaf(fmaf(a, c.c4, c.c3), a, c.c2) : fmaf(a, c.c3, c.c2);
+    t = fmaf(a, t, c.c1);
+    t = fmaf(a, t, 1.0f);
+    return fmaf(pp * a, t, S);
 }
 
 constexpr int kHeadWarps = 4;   // tokens per block
@@ -96,8 +107,9 @@ head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
                   float* __restrict__ g, __nv_bfloat16* __restrict__ g16, int accumulate) {
     constexpr int kTPB = kHeadWarps / WPT;        // tokens per block
     constexpr int kSub = 128 * QPL;               // vocab ids per warp
-    // the softmax probabilities of each warp's ids: read every draw, so they
-    // live in shared memory and leave the registers to a and g
+    // the softmax probabilities of each warp's ids (times sigma for the series
+    // tiers): read every draw, so they live in shared memory and leave the
+    // registers to a and g
     __shared__ float4 p_s[kHeadWarps][32 * QPL];
     __shared__ float red_s[kTPB][2][WPT], red_ay[kTPB][2][WPT];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -109,10 +121,13 @@ head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
     const float* zt = Z + static_cast<size_t>(t) * V;
     const float l = __ldg(lse + t);
     float4* p = p_s[warp];
+    const float ps = TIER == 0 ? 1.0f : sigma;
+    const ExpCoef ec = exp_coef(sigma);
 #pragma unroll
     for (int k = 0; k < QPL; ++k) {
         const float4 z = __ldg(reinterpret_cast<const float4*>(zt + v0 + 4 * (lane + 32 * k)));
-        p[lane + 32 * k] = make_float4(expf(z.x - l), expf(z.y - l), expf(z.z - l), expf(z.w - l));
+        p[lane + 32 * k] =
+            make_float4(ps * expf(z.x - l), ps * expf(z.y - l), ps * expf(z.z - l), ps * expf(z.w - l));
     }
     __syncwarp();
     const int rel_chunk = clamp_int(__ldg(targets + t), 0, V - 1) - chunk * Vc;
@@ -140,10 +155,7 @@ head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
             const float4 pk = p[lane + 32 * k];
             const float pv[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const float x = sigma * a[k][w];
-                S = fmaf(pv[w], TIER == 0 ? expm1f(x) : expm1_series<TIER>(x), S);
-            }
+            for (int w = 0; w < 4; ++w) S = add_p_expm1<TIER>(S, pv[w], a[k][w], sigma, ec);
             if (i_own && k == ky) ay = wy == 0 ? n.x : (wy == 1 ? n.y : (wy == 2 ? n.z : n.w));
         }
         S = warp_sum(S);

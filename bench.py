@@ -373,7 +373,8 @@ def launches_per_step(step):
 
 def load_traffic():
     """ncu DRAM bytes per output unit from profiles/traffic.txt, for kernels whose
-    source is unchanged since the capture (sha1 prefix match); else absent."""
+    source files ('+'-joined, hashed in order) are unchanged since the capture
+    (sha1 prefix match); else absent."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     out = {}
@@ -383,10 +384,13 @@ def load_traffic():
         if ln.startswith("#") or not ln.strip():
             continue
         kernel, per_unit, unit, src, sha = ln.split()
+        h = hashlib.sha1()
         try:
-            cur = hashlib.sha1(open(os.path.join(ROOT, src), "rb").read()).hexdigest()[:len(sha)]
+            for f in src.split("+"):          # the kernel's file and the headers it inlines
+                h.update(open(os.path.join(ROOT, f), "rb").read())
         except OSError:
             continue
+        cur = h.hexdigest()[:len(sha)]
         if cur == sha:
             out[kernel] = (float(per_unit), unit)
     return out
