@@ -82,14 +82,17 @@ __device__ __forceinline__ ExpCoef exp_coef(float sigma) {
             sigma * sigma * sigma * sigma * (1.0f / 120.0f)};
 }
 
-// S + p expm1(sigma a); pp is p (tier 0) or p sigma (series tiers)
+// S + p expm1(sigma a) on two packed lanes; pp is p (tier 0) or p sigma
+// (series tiers)
 template <int TIER>
-__device__ __forceinline__ float add_p_expm1(float S, float pp, float a, float sigma, const ExpCoef& c) {
-    if (TIER == 0) return fmaf(pp, expm1f(sigma * a), S);
-    float t = TIER == 1 ? fmaf(fmaf(a, c.c4, c.c3), a, c.c2) : fmaf(a, c.c3, c.c2);
-    t = fmaf(a, t, c.c1);
-    t = fmaf(a, t, 1.0f);
-    return fmaf(pp * a, t, S);
+__device__ __forceinline__ float2 add_p_expm1(float2 S, float2 pp, float2 a, float sigma, const ExpCoef& c) {
+    if (TIER == 0)
+        return make_float2(fmaf(pp.x, expm1f(sigma * a.x), S.x), fmaf(pp.y, expm1f(sigma * a.y), S.y));
+    float2 t = TIER == 1 ? __ffma2_rn(__ffma2_rn(a, splat(c.c4), splat(c.c3)), a, splat(c.c2))
+                         : __ffma2_rn(a, splat(c.c3), splat(c.c2));
+    t = __ffma2_rn(a, t, splat(c.c1));
+    t = __ffma2_rn(a, t, splat(1.0f));
+    return __ffma2_rn(__fmul2_rn(pp, a), t, S);
 }
 
 constexpr int kHeadWarps = 4;   // tokens per block
@@ -109,7 +112,8 @@ head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
     constexpr int kSub = 128 * QPL;               // vocab ids per warp
     // the softmax probabilities of each warp's ids (times sigma for the series
     // tiers): read every draw, so they live in shared memory and leave the
-    // registers to a and g
+    // registers to a and g.  Each quad is stored as (p0, p2, p1, p3), the
+    // even- and odd-channel lanes of the packed arithmetic.
     __shared__ float4 p_s[kHeadWarps][32 * QPL];
     __shared__ float red_s[kTPB][2][WPT], red_ay[kTPB][2][WPT];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -127,7 +131,7 @@ head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
     for (int k = 0; k < QPL; ++k) {
         const float4 z = __ldg(reinterpret_cast<const float4*>(zt + v0 + 4 * (lane + 32 * k)));
         p[lane + 32 * k] =
-            make_float4(ps * expf(z.x - l), ps * expf(z.y - l), ps * expf(z.z - l), ps * expf(z.w - l));
+            make_float4(ps * expf(z.x - l), ps * expf(z.z - l), ps * expf(z.y - l), ps * expf(z.w - l));
     }
     __syncwarp();
     const int rel_chunk = clamp_int(__ldg(targets + t), 0, V - 1) - chunk * Vc;
@@ -139,25 +143,27 @@ head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
     const int wy = rel & 3;
     const bool i_own = in_mine && lane == owner;
 
-    float gacc[QPL][4];
+    float2 ge[QPL], go[QPL];      // g of the even channels (4q, 4q+2) and the odd ones (4q+1, 4q+3)
 #pragma unroll
-    for (int k = 0; k < QPL; ++k) gacc[k][0] = gacc[k][1] = gacc[k][2] = gacc[k][3] = 0.0f;
+    for (int k = 0; k < QPL; ++k) ge[k] = go[k] = splat(0.0f);
     const uint32_t quad0 = static_cast<uint32_t>(v0 / 4 + lane);
 
     for (int i = 0; i < nd; ++i) {
         const uint32_t draw = draw_begin + static_cast<uint32_t>(i);
-        float a[QPL][4];
-        float S = 0.0f, ay = 0.0f;
+        float2 ae[QPL], ao[QPL];
+        float2 S2 = splat(0.0f);
+        float ay = 0.0f;
 #pragma unroll
         for (int k = 0; k < QPL; ++k) {
-            const float4 n = gauss4(seed, layer, draw, static_cast<uint32_t>(t), quad0 + 32u * k, 0);
-            a[k][0] = n.x; a[k][1] = n.y; a[k][2] = n.z; a[k][3] = n.w;
+            const Gauss4Pairs n = gauss4_pairs(seed, layer, draw, static_cast<uint32_t>(t), quad0 + 32u * k, 0);
+            ae[k] = n.even;
+            ao[k] = n.odd;
             const float4 pk = p[lane + 32 * k];
-            const float pv[4] = {pk.x, pk.y, pk.z, pk.w};
-#pragma unroll
-            for (int w = 0; w < 4; ++w) S = add_p_expm1<TIER>(S, pv[w], a[k][w], sigma, ec);
-            if (i_own && k == ky) ay = wy == 0 ? n.x : (wy == 1 ? n.y : (wy == 2 ? n.z : n.w));
+            S2 = add_p_expm1<TIER>(S2, make_float2(pk.x, pk.y), ae[k], sigma, ec);
+            S2 = add_p_expm1<TIER>(S2, make_float2(pk.z, pk.w), ao[k], sigma, ec);
+            if (i_own && k == ky) ay = wy == 0 ? ae[k].x : (wy == 1 ? ao[k].x : (wy == 2 ? ae[k].y : ao[k].y));
         }
+        float S = S2.x + S2.y;
         S = warp_sum(S);
         ay = __shfl_sync(0xffffffffu, ay, owner);      // 0 unless this warp holds the target
         float sy = in_mine ? sigma * ay : 0.0f;
@@ -178,16 +184,18 @@ head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
         }
         const float c = log1pf(S) - (in_chunk ? sy : 0.0f);
         if (c_out != nullptr && lane == 0 && part == 0) c_out[(static_cast<size_t>(chunk) * nd + i) * T + t] = c;
+        const float2 cc = splat(c);
 #pragma unroll
-        for (int k = 0; k < QPL; ++k)
-#pragma unroll
-            for (int w = 0; w < 4; ++w) gacc[k][w] = fmaf(c, a[k][w], gacc[k][w]);
+        for (int k = 0; k < QPL; ++k) {
+            ge[k] = __ffma2_rn(cc, ae[k], ge[k]);
+            go[k] = __ffma2_rn(cc, ao[k], go[k]);
+        }
     }
 
 #pragma unroll
     for (int k = 0; k < QPL; ++k) {
         const size_t off = static_cast<size_t>(t) * V + v0 + 4 * (lane + 32 * k);
-        float4 out = make_float4(gacc[k][0] * scale, gacc[k][1] * scale, gacc[k][2] * scale, gacc[k][3] * scale);
+        float4 out = make_float4(ge[k].x * scale, go[k].x * scale, ge[k].y * scale, go[k].y * scale);
         float4* gp = reinterpret_cast<float4*>(g + off);
         if (accumulate) {
             const float4 o = *gp;

@@ -9,7 +9,8 @@
 // stored, and the only HBM traffic is r (4 bytes per draw x token, a warp-wide
 // broadcast) and g (written once).  The kernel is therefore bound by the SM
 // issue rate, not by HBM.  One thread owns (token t, channel quad q): a single
-// Philox call per draw yields its 4 channels, so the counter words that do not
+// Philox call per draw yields its 4 channels, whose two Box-Muller pairs run
+// in lock-step on the packed fp32 pipes, so the counter words that do not
 // depend on the draw (first-round product of the quad, key schedule) are
 // hoisted out of the draw loop.  Two draws per iteration give the scheduler two
 // independent Philox chains.  Blocks are 256 threads: quads along x (coalesced
@@ -24,18 +25,17 @@ namespace dust {
 
 namespace {
 
-// acc += r * a for the 4 channels of one Philox call; r is folded into the
-// Box-Muller radius (r * rho once per pair instead of rho * cos and rho * sin).
-__device__ __forceinline__ void accumulate_quad(float4& acc, float r, uint32_t seed, uint32_t layer, uint32_t draw,
-                                                uint32_t token, uint32_t quad) {
+// acc += r * a for the 4 channels of one Philox call, as two packed lanes:
+// xz holds channels (4q, 4q+2), yw channels (4q+1, 4q+3).  r is folded into
+// the Box-Muller radius (r * rho once per pair instead of rho * cos and
+// rho * sin).
+__device__ __forceinline__ void accumulate_quad(float2& xz, float2& yw, float r, uint32_t seed, uint32_t layer,
+                                                uint32_t draw, uint32_t token, uint32_t quad) {
     const uint4 x = philox4x32_10(make_uint4(quad, token, draw, 0u), seed, layer);
-    const Polar p01 = box_muller_polar(x.x, x.y);
-    const Polar p23 = box_muller_polar(x.z, x.w);
-    const float r01 = r * p01.rho, r23 = r * p23.rho;
-    acc.x = __fmaf_rn(r01, p01.cos_t, acc.x);
-    acc.y = __fmaf_rn(r01, p01.sin_t, acc.y);
-    acc.z = __fmaf_rn(r23, p23.cos_t, acc.z);
-    acc.w = __fmaf_rn(r23, p23.sin_t, acc.w);
+    const Polar2 p = box_muller_polar2(x.x, x.y, x.z, x.w);
+    const float2 rr = __fmul2_rn(splat(r), p.rho);
+    xz = __ffma2_rn(rr, p.cos_t, xz);
+    yw = __ffma2_rn(rr, p.sin_t, yw);
 }
 
 // The epilogue's options are template parameters (kVec: d_out % 4 == 0, 128-bit
@@ -49,22 +49,21 @@ layer_estimate_kernel(const float* __restrict__ r, int T, int d_out, int nq, uin
     const int q = blockIdx.x * blockDim.x + threadIdx.x;
     if (q >= nq) return;
     for (int t = blockIdx.y * blockDim.y + threadIdx.y; t < T; t += gridDim.y * blockDim.y) {
-        float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f);
-        float4 acc1 = make_float4(0.f, 0.f, 0.f, 0.f);
+        float2 xz0 = splat(0.0f), yw0 = splat(0.0f), xz1 = splat(0.0f), yw1 = splat(0.0f);
         const float* rt = r + t;
         int k = 0;
         for (; k + 2 <= nd; k += 2) {
             const float r0 = __ldg(rt + static_cast<size_t>(k) * T);
             const float r1 = __ldg(rt + static_cast<size_t>(k + 1) * T);
-            accumulate_quad(acc0, r0, seed, layer, draw_begin + k, t, q);
-            accumulate_quad(acc1, r1, seed, layer, draw_begin + k + 1, t, q);
+            accumulate_quad(xz0, yw0, r0, seed, layer, draw_begin + k, t, q);
+            accumulate_quad(xz1, yw1, r1, seed, layer, draw_begin + k + 1, t, q);
         }
         if (k < nd) {
             const float r0 = __ldg(rt + static_cast<size_t>(k) * T);
-            accumulate_quad(acc0, r0, seed, layer, draw_begin + k, t, q);
+            accumulate_quad(xz0, yw0, r0, seed, layer, draw_begin + k, t, q);
         }
-        float4 out = make_float4((acc0.x + acc1.x) * scale, (acc0.y + acc1.y) * scale,
-                                 (acc0.z + acc1.z) * scale, (acc0.w + acc1.w) * scale);
+        float4 out = make_float4((xz0.x + xz1.x) * scale, (yw0.x + yw1.x) * scale,
+                                 (xz0.y + xz1.y) * scale, (yw0.y + yw1.y) * scale);
         const size_t base = static_cast<size_t>(t) * d_out + 4 * static_cast<size_t>(q);
         if constexpr (kVec) {
             float4* gp = reinterpret_cast<float4*>(g + base);

@@ -30,13 +30,23 @@ __global__ void noise_fill_kernel(uint32_t seed, uint32_t layer, uint32_t stream
     }
 }
 
+// For n = 2h (+1): element i < h runs in lane .x and element i + h in lane .y
+// of the packed generator (the one the hot kernels inline); an odd last
+// element n - 1 runs in lane .x with a copy of itself in lane .y.
 __global__ void box_muller_words_kernel(const uint32_t* __restrict__ a, const uint32_t* __restrict__ b, long long n,
                                         float* __restrict__ ne, float* __restrict__ no) {
-    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+    const long long h = n >> 1, pairs = (n + 1) >> 1;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < pairs;
          i += static_cast<long long>(gridDim.x) * blockDim.x) {
-        const float2 v = box_muller(a[i], b[i]);
-        ne[i] = v.x;
-        no[i] = v.y;
+        const long long i0 = i < h ? i : n - 1, i1 = i < h ? i + h : n - 1;
+        const Polar2 p = box_muller_polar2(a[i0], b[i0], a[i1], b[i1]);
+        const float2 e = __fmul2_rn(p.rho, p.cos_t), o = __fmul2_rn(p.rho, p.sin_t);
+        ne[i0] = e.x;
+        no[i0] = o.x;
+        if (i1 != i0) {
+            ne[i1] = e.y;
+            no[i1] = o.y;
+        }
     }
 }
 
@@ -99,7 +109,7 @@ cudaError_t launch_noise_fill(const dust_noise& nz, uint32_t stream_id, int t0, 
 cudaError_t launch_box_muller_words(const uint32_t* a, const uint32_t* b, long long n, float* ne, float* no,
                                     cudaStream_t stream) {
     if (n == 0) return cudaSuccess;
-    const long long blocks = ceil_div(n, 256);
+    const long long blocks = ceil_div((n + 1) / 2, 256);
     box_muller_words_kernel<<<static_cast<unsigned>(blocks < 8 * 1184 ? blocks : 8 * 1184), 256, 0, stream>>>(a, b, n,
                                                                                                             ne, no);
     return cudaGetLastError();

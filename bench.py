@@ -41,17 +41,29 @@ DEFAULT_WORKLOAD = I.SCALED.name
 METRIC = "Dust draws×tokens/s per layer step"
 UNIT = "draws×tokens/s"
 
-# Algorithmic work per element of the ALU-bound kernels, counted from the
-# operation sequence of the noise specification (one lane-operation per
-# primitive: integer mul-hi/lo, xor, shift, and/or, add, select; fp add, mul,
-# fma, div, sqrt; an exp-family function counts as one).
-#   Philox4x32-10: 10 rounds x (2 wide products = 4, 4 xors) = 80 per 4 Gaussians -> 20
-#   Box-Muller pair: uniforms 3, ln 18, rho 2, angle 8, sin/cos 12, octant
-#   swap 5, signs 8, products 2 = 58 per 2 Gaussians -> 29
-OPS_PER_GAUSSIAN = 49
-OPS_A5 = OPS_PER_GAUSSIAN + 1          # + the FMA into g
-OPS_HEAD = OPS_PER_GAUSSIAN + 4        # + sigma*a, expm1, FMA into S, FMA into g
-LANES_PER_SM = 128
+# Algorithmic work per element of the ALU-bound kernels, in lane issue slots:
+# the noise specification's operations, each in its cheapest sm_100 instruction
+# form (one warp instruction issues per scheduler per clock, so a lane gets one
+# slot per clock).  Counted per Philox call (4 elements, 2 Box-Muller pairs):
+#   Philox4x32-10: 10 rounds x (2 wide 32x32->64 products + 2 three-input xors),
+#     less the draw-independent product and xor of round 1              = 38
+#   radius uniforms: 2 shift-and-insert + 1 packed subtraction          =  3
+#   ln: 2 x 4 integer (exponent split, magic float) + 15 packed fp32
+#     (4(m-1), m+1, quotient correction 3, square, Horner 5, product, magic,
+#     2 fma) + 2 reciprocal estimates                                   = 25
+#   sqrt: 2 clamps + 2 reciprocal-sqrt estimates + 4 packed             =  8
+#   angle: 2 x 2 fraction bits + 4 packed + 2 x 2 odd-octant select     = 12
+#   sin / cos Horner: 11 packed                                         = 11
+#   octant swap and signs: 2 x 7                                        = 14
+# (packed: one __ffma2_rn / __fadd2_rn / __fmul2_rn for the same fp32 op on
+# both pairs).  Consumers: the hidden reduction adds r rho and two fma (3
+# packed) and the load of r (1) = 4; the head adds a = rho cos / rho sin (2),
+# the expm1 series and the sum (10), the fma into g (2) and the load of p (1)
+# = 15.  Not counted (so the bound stays an upper bound): loop control, the
+# head's per-draw warp reduction and log1p.
+SLOTS_A5 = (111 + 4) / 4               # 28.75 per Gaussian
+SLOTS_HEAD = (111 + 15) / 4            # 31.5 per perturbed logit
+LANES_PER_SM = 128                     # 4 schedulers x 32 lanes
 
 
 def parse_args():
@@ -399,7 +411,7 @@ def load_traffic():
 def kernel_report(step, stages, peaks, clocks):
     w, K, T = step.w, step.K, step.w.T
     f_peak = peaks["sm_max_mhz"]
-    alu_peak = 148 * LANES_PER_SM * f_peak * 1e6 / 1e12          # Tops/s
+    alu_peak = 148 * LANES_PER_SM * f_peak * 1e6 / 1e12          # T lane-slots/s
     out = []
     names = step.stage_names
     traffic = load_traffic()
@@ -422,19 +434,21 @@ def kernel_report(step, stages, peaks, clocks):
             rec |= {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                     "frac": ach / peaks["bf16_tflops"], "traffic": None, "algorithmic_flops": fl}
         else:
-            ops_el = OPS_HEAD if layer == "head" else OPS_A5
-            ops = float(K) * T * d_out * ops_el
-            ach = ops / (ms / 1e3) / 1e12
+            slots_el = SLOTS_HEAD if layer == "head" else SLOTS_A5
+            slots = float(K) * T * d_out * slots_el
+            ach = slots / (ms / 1e3) / 1e12
             tkey = "head_chunk_kernel" if layer == "head" else "layer_estimate"
             tr = traffic.get(tkey)
-            rec |= {"bound": "alu", "achieved": ach, "peak": alu_peak, "unit": "Tops/s",
+            rec |= {"bound": "alu", "achieved": ach, "peak": alu_peak, "unit": "T lane-slots/s",
                     "frac": ach / alu_peak, "traffic": tr[0] * T * d_out if tr else None,
                     "traffic_source": "profiles/traffic.txt (ncu small case, scaled by tokens x channels)"
                     if tr else None,
-                    "algorithmic_ops": ops,
-                    "ops_per_element": ops_el, "clock_mhz_for_peak": f_peak,
+                    "algorithmic_slots": slots,
+                    "slots_per_element": slots_el, "clock_mhz_for_peak": f_peak,
                     "gaussians_per_s": float(K) * T * d_out / (ms / 1e3),
-                    "peak_source": "148 SMs x 128 lanes x max SM clock (one lane-op per lane per clock)"}
+                    "peak_source": "148 SMs x 4 schedulers x 32 lanes x max SM clock (one issue slot per lane "
+                                   "per clock); work = the specification's operations in their cheapest sm_100 "
+                                   "instruction forms"}
         out.append(rec)
     return out
 
