@@ -247,6 +247,70 @@ dust_status dust_layer_estimate(const float* c_or_r, int is_r, int T, int d_out,
                        "dust_layer_estimate");
 }
 
+// ------------------------------------------------------------------ a1 + a5 + a6 fused
+namespace {
+struct FusedWs {
+    size_t r_off = 0, chunk_off = 0, part_off = 0, total = 0;
+    bool scan = false;
+};
+
+FusedWs fused_ws(int K, int T, int d_in, int d_out, int is_r, float gamma) {
+    FusedWs w;
+    Layout L;
+    w.scan = !is_r && gamma != 0.0f;
+    if (w.scan) {
+        w.r_off = L.add(sizeof(float) * static_cast<size_t>(K) * T);
+        w.chunk_off = L.add(dust::reward_scan_chunks_workspace(K, T));
+    }
+    w.part_off = L.add(dust::fused_estimate_scratch(T, d_in, d_out));
+    w.total = L.off;
+    return w;
+}
+}  // namespace
+
+size_t dust_layer_estimate_weight_grad_workspace(int draw_count, int T, int d_in, int d_out, int is_r, float gamma) {
+    if (draw_count <= 0 || T <= 0 || !dust::fused_estimate_supported(d_in, d_out)) return dust::kStatusBytes;
+    return fused_ws(draw_count, T, d_in, d_out, is_r, gamma).total;
+}
+
+dust_status dust_layer_estimate_weight_grad(const float* c_or_r, int is_r, int T, int d_out,
+                                            const int32_t* seq_offsets, int n_seq, float gamma, dust_noise nz,
+                                            const void* X, int d_in, float* G_W, int accumulate, float* g_hat_out,
+                                            void* ws, size_t ws_bytes, void* stream) {
+    DUST_TRY(check_noise(nz));
+    DUST_REQUIRE(T > 0 && d_out > 0, DUST_ERR_INVALID_ARG, "T and d_out must be > 0 (T=%d, d_out=%d)", T, d_out);
+    DUST_REQUIRE(dust::fused_estimate_supported(d_in, d_out), DUST_ERR_UNSUPPORTED,
+                 "d_in must be a multiple of 64 in [64, 512] (d_in=%d)", d_in);
+    DUST_REQUIRE(std::isfinite(gamma) && gamma >= 0.0f && gamma <= 1.0f, DUST_ERR_INVALID_ARG,
+                 "gamma must be in [0, 1]");
+    DUST_REQUIRE(static_cast<long long>(nz.draw_count) * T < (1ll << 31), DUST_ERR_INVALID_ARG,
+                 "draw_count x T must be < 2^31");
+    DUST_TRY(check_ptr(c_or_r, "c_or_r"));
+    DUST_TRY(check_ptr(X, "X"));
+    DUST_TRY(check_ptr(G_W, "G_W"));
+    DUST_TRY(check_ptr(g_hat_out, "g_hat_out", true));
+    DUST_TRY(check_ptr(ws, "ws"));
+    const int K = static_cast<int>(nz.draw_count);
+    const FusedWs w = fused_ws(K, T, d_in, d_out, is_r, gamma);
+    DUST_REQUIRE(ws_bytes >= w.total, DUST_ERR_WORKSPACE, "workspace %zu bytes < %zu", ws_bytes, w.total);
+    cudaStream_t st = as_stream(stream);
+    const float* r = c_or_r;
+    if (w.scan) {
+        DUST_TRY(check_seq(seq_offsets, n_seq, K, T));
+        float* rw = reinterpret_cast<float*>(region(ws, w.r_off));
+        const cudaError_t e = dust::reward_scan_prefers_chunks(K, T, n_seq)
+                                  ? dust::launch_reward_scan_chunks(c_or_r, rw, K, T, seq_offsets, n_seq, gamma,
+                                                                    region(ws, w.chunk_off), st)
+                                  : dust::launch_reward_scan(c_or_r, rw, K, T, seq_offsets, n_seq, gamma, st);
+        DUST_TRY(cuda_status(e, "dust_layer_estimate_weight_grad (scan)"));
+        r = rw;
+    }
+    const cudaError_t e = dust::launch_fused_estimate(r, T, d_out, X, d_in, nz, G_W, accumulate, g_hat_out,
+                                                      region(ws, w.part_off), static_cast<uint32_t*>(ws), st);
+    DUST_REQUIRE(e != cudaErrorNotSupported, DUST_ERR_UNSUPPORTED, "shape not supported by the fused kernel");
+    return cuda_status(e, "dust_layer_estimate_weight_grad");
+}
+
 // ------------------------------------------------------------------ a6
 static GemmPlan weight_grad_plan(int T, int d_in, int d_out, dust_dtype dt) {
     // C[d_out][d_in] = sum_t g[t][o] X[t][i]: A = g (M-major), B = X (N-major)

@@ -2,6 +2,7 @@
 // `stream` and returns the launch status; argument validation happens in
 // api.cu before any of these is called.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -57,6 +58,20 @@ cudaError_t launch_gemm_tc(const void* A, bool a_kmajor, int lda, const void* B,
 int gemm_tc_splits(int M, int N, int K);
 cudaError_t launch_bounded_wait_selftest(uint32_t* status, uint32_t polls, cudaStream_t stream);
 bool gemm_tc_supported(int M, int N, int K, bool a_kmajor, bool b_kmajor);
+// 2-D bf16 tensor map [outer][inner], row pitch ld elements, box {64, box_outer},
+// 128-byte swizzle; false when the driver entry point or the encoding fails
+bool tma_map_bf16_2d(CUtensorMap* map, const void* base, int inner, int outer, int ld, int box_outer);
+int device_sm_count();
+
+// a1 + a5 + a6 fused (fused_estimate.cu): G (+)= sum_t bf16(g_t) x_t^T with g
+// produced in shared memory (never written unless g_hat is given);
+// d_in a multiple of 64 up to 512.  scratch holds fused_estimate_scratch()
+// bytes (fp32 partial G row blocks, one per token split).
+bool fused_estimate_supported(int d_in, int d_out);
+size_t fused_estimate_scratch(int T, int d_in, int d_out);
+cudaError_t launch_fused_estimate(const float* r, int T, int d_out, const void* X, int d_in, const dust_noise& nz,
+                                  float* G, int accumulate, float* g_hat, void* scratch, uint32_t* status,
+                                  cudaStream_t stream);
 
 // a2 row statistics + a3/a5 fused head (head.cu)
 cudaError_t launch_row_stats(const float* Z, const int32_t* targets, int T, int V, float* lse,

@@ -19,24 +19,12 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "estimate.cuh"
 #include "noise.cuh"
 
 namespace dust {
 
 namespace {
-
-// acc += r * a for the 4 channels of one Philox call, as two packed lanes:
-// xz holds channels (4q, 4q+2), yw channels (4q+1, 4q+3).  r is folded into
-// the Box-Muller radius (r * rho once per pair instead of rho * cos and
-// rho * sin).
-__device__ __forceinline__ void accumulate_quad(float2& xz, float2& yw, float r, uint32_t seed, uint32_t layer,
-                                                uint32_t draw, uint32_t token, uint32_t quad) {
-    const uint4 x = philox4x32_10(make_uint4(quad, token, draw, 0u), seed, layer);
-    const Polar2 p = box_muller_polar2(x.x, x.y, x.z, x.w);
-    const float2 rr = __fmul2_rn(splat(r), p.rho);
-    xz = __ffma2_rn(rr, p.cos_t, xz);
-    yw = __ffma2_rn(rr, p.sin_t, yw);
-}
 
 // The epilogue's options are template parameters (kVec: d_out % 4 == 0, 128-bit
 // stores; kAcc: add into g; kG16: also write the bf16 copy): with runtime flags

@@ -65,6 +65,9 @@ _SIGS = {
     "dust_layer_estimate": ([_vp, _i, _i, _i, _vp, _i, _f, _Noise, _vp, _vp, _i, _vp, _sz, _vp], _i),
     "dust_layer_estimate_workspace": ([_i, _i, _i, _i, _f], _sz),
     "dust_layer_estimate_noalloc": ([_vp, _i, _i, _vp, _i, _f, _Noise, _vp, _vp, _i, _vp], _i),
+    "dust_layer_estimate_weight_grad": ([_vp, _i, _i, _i, _vp, _i, _f, _Noise, _vp, _i, _vp, _i, _vp, _vp, _sz, _vp],
+                                        _i),
+    "dust_layer_estimate_weight_grad_workspace": ([_i, _i, _i, _i, _i, _f], _sz),
     "dust_weight_grad": ([_vp, _vp, _i, _i, _i, _i, _vp, _i, _vp, _sz, _vp], _i),
     "dust_weight_grad_workspace": ([_i, _i, _i, _i], _sz),
     "dust_logits": ([_vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp], _i),
@@ -212,6 +215,36 @@ def layer_estimate(c_or_r: torch.Tensor, is_r: bool, seq_offsets, gamma: float, 
                                      _opt(g_hat_bf16, "g_hat_bf16", torch.bfloat16), int(bool(accumulate)),
                                      ws.data_ptr(), ws.numel(), _stream()))
     return g_hat, g_hat_bf16
+
+
+def layer_estimate_weight_grad(c_or_r: torch.Tensor, is_r: bool, seq_offsets, gamma: float, noise: Noise,
+                               X: torch.Tensor, d_out: int, G_W: torch.Tensor | None = None, accumulate: bool = False,
+                               g_hat: torch.Tensor | bool | None = None):
+    """dust_layer_estimate_weight_grad: G_W [d_out][d_in] fp32 from costs or
+    rewards and bf16 X [T][d_in] in one fused pass (g never leaves the chip).
+    g_hat=True (or a tensor) also returns g. Returns (G_W, g_hat or None)."""
+    nd, T = c_or_r.shape
+    if nd != noise.draw_count:
+        raise ValueError("c_or_r must have draw_count rows")
+    if X.dim() != 2 or X.shape[0] != T:
+        raise ValueError("X must be [T][d_in]")
+    d_in = X.shape[1]
+    dev = c_or_r.device
+    if G_W is None:
+        G_W = torch.empty(d_out, d_in, dtype=torch.float32, device=dev)
+    if g_hat is True:
+        g_hat = torch.empty(T, d_out, dtype=torch.float32, device=dev)
+    elif g_hat is False:
+        g_hat = None
+    need = lib().dust_layer_estimate_weight_grad_workspace(nd, T, d_in, d_out, int(bool(is_r)), float(gamma))
+    ws = workspace(need, dev)
+    offs = None if seq_offsets is None else _dev(seq_offsets, "seq_offsets", torch.int32)
+    n_seq = 1 if seq_offsets is None else seq_offsets.numel() - 1
+    _check(lib().dust_layer_estimate_weight_grad(
+        _dev(c_or_r, "c_or_r", torch.float32), int(bool(is_r)), T, d_out, offs, n_seq, float(gamma), noise.c(),
+        _dev(X, "X", torch.bfloat16), d_in, _dev(G_W, "G_W", torch.float32), int(bool(accumulate)),
+        _opt(g_hat, "g_hat", torch.float32), ws.data_ptr(), ws.numel(), _stream()))
+    return G_W, g_hat
 
 
 def layer_estimate_noalloc(c: torch.Tensor, seq_offsets, gamma: float, noise: Noise, d_out: int,

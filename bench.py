@@ -76,6 +76,9 @@ def parse_args():
     p.add_argument("--draws", type=int, default=0, help="override the workload's K")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--fused", action="store_true",
+                   help="hidden layers with d_in a multiple of 64 up to 512 run the draw reduction and the weight "
+                        "estimate as one kernel (dust_layer_estimate_weight_grad)")
     return p.parse_args()
 
 
@@ -183,7 +186,7 @@ def max_over_ranks(x, world):
 class Step:
     """Device-resident buffers and the sequence of C-ABI calls of one step."""
 
-    def __init__(self, w: I.Workload, K: int, rank: int, world: int):
+    def __init__(self, w: I.Workload, K: int, rank: int, world: int, fused: bool = False):
         import torch
         from activation_perturbation_es_b200 import dust
         self.torch, self.dust, self.w, self.K, self.world = torch, dust, w, K, world
@@ -202,6 +205,7 @@ class Step:
             del u
             X = torch.from_numpy(li["X"]).to(dev, bf)
             L = {"hl": hl, "nz": nz, "c": c, "X": X,
+                 "fused": fused and hl.d_in % 64 == 0 and 64 <= hl.d_in <= 512,
                  "r": torch.empty_like(c),
                  "g": torch.empty(T, hl.d_out, dtype=torch.float32, device=dev),
                  "g16": torch.empty(T, hl.d_out, dtype=bf, device=dev),
@@ -222,7 +226,8 @@ class Step:
         self.stage_names = []
         for L in self.hidden:
             n = L["hl"].name
-            self.stage_names += [f"{n}:scan", f"{n}:estimate", f"{n}:weight_grad"]
+            self.stage_names += [f"{n}:scan"] + ([f"{n}:fused_estimate_wgrad"] if L["fused"]
+                                                 else [f"{n}:estimate", f"{n}:weight_grad"])
         if self.head:
             self.stage_names += ["head:logits", "head:ce_estimate", "head:weight_grad"]
         self.events = None
@@ -250,10 +255,10 @@ class Step:
             mark()
             dust.reward_scan(L["c"], self.off, self.w.gamma, out=L["r"])
             mark()
-            dust.layer_estimate(L["r"], True, self.off, self.w.gamma, L["nz"], hl.d_out, g_hat=L["g"],
-                                g_hat_bf16=L["g16"])
-            mark()
-            dust.weight_grad(L["g16"], L["X"], G_W=L["G"])
+            self._estimate(L)
+            if not L["fused"]:
+                mark()
+                dust.weight_grad(L["g16"], L["X"], G_W=L["G"])
         if self.head:
             H = self.head
             mark()
@@ -274,11 +279,10 @@ class Step:
         for L in self.hidden:
             cur.wait_event(ready[j])
             j += 1
-            hl = L["hl"]
             dust.reward_scan(L["c"], self.off, self.w.gamma, out=L["r"])
-            dust.layer_estimate(L["r"], True, self.off, self.w.gamma, L["nz"], hl.d_out, g_hat=L["g"],
-                                g_hat_bf16=L["g16"])
-            dust.weight_grad(L["g16"], L["X"], G_W=L["G"])
+            self._estimate(L)
+            if not L["fused"]:
+                dust.weight_grad(L["g16"], L["X"], G_W=L["G"])
         if self.head:
             H = self.head
             cur.wait_event(ready[j])
@@ -287,6 +291,16 @@ class Step:
             dust.weight_grad(H["g16"], H["X"], G_W=H["G"])
         if self.world > 1:
             self.allreduce()
+
+    def _estimate(self, L):
+        """The draw reduction; fused with the weight estimate when L is eligible."""
+        hl = L["hl"]
+        if L["fused"]:
+            self.dust.layer_estimate_weight_grad(L["r"], True, self.off, self.w.gamma, L["nz"], L["X"], hl.d_out,
+                                                 G_W=L["G"])
+        else:
+            self.dust.layer_estimate(L["r"], True, self.off, self.w.gamma, L["nz"], hl.d_out, g_hat=L["g"],
+                                     g_hat_bf16=L["g16"])
 
     def allreduce(self):
         from activation_perturbation_es_b200 import dp
@@ -311,7 +325,7 @@ def main():
     w = I.WORKLOADS[args.workload]
     K = args.draws or w.K
     peaks = load_peaks()
-    step = Step(w, K, rank, world)
+    step = Step(w, K, rank, world, fused=args.fused)
     for _ in range(args.warmup):
         step.run()
     torch.cuda.synchronize()
@@ -352,6 +366,7 @@ def main():
                        "hidden": [[h.d_in, h.d_out] for h in w.hidden],
                        "head": {"d": w.head_d, "V": w.V, "Vc": w.Vc} if w.V else None,
                        "parallelism": f"dp{world}", "l2": "inputs larger than L2 (126 MB); no flush",
+                       "fused_estimate_wgrad": bool(args.fused),
                        "arithmetic": "f32 noise, cross entropy and reductions; bf16 GEMM operands with f32 "
                                      "accumulation in TMEM (tcgen05)"},
             "roofline": {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
@@ -374,6 +389,9 @@ def launches_per_step(step):
     n = 0
     for L in step.hidden:
         n += 1                                   # reward scan
+        if L["fused"]:
+            n += 2                               # fused reduction + weight GEMM, split reduction
+            continue
         n += 1                                   # draw reduction
         n += 1 if step.dust.lib().dust_weight_grad_workspace(step.w.T, L["hl"].d_in, L["hl"].d_out, 1) <= 256 else 2
     if step.head:
@@ -428,6 +446,17 @@ def kernel_report(step, stages, peaks, clocks):
             ach = byts / (ms / 1e3) / 1e9
             rec |= {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": ach / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes": byts}
+        elif kind == "fused_estimate_wgrad":
+            # ALU-bound like the reduction it contains; the GEMM's flops ride on the tensor pipe alongside
+            slots = float(K) * T * d_out * SLOTS_A5
+            ach = slots / (ms / 1e3) / 1e12
+            f_peak = peaks["sm_max_mhz"]
+            rec |= {"bound": "alu", "achieved": ach, "peak": alu_peak, "unit": "T lane-slots/s",
+                    "frac": ach / alu_peak, "traffic": None, "algorithmic_slots": slots,
+                    "slots_per_element": SLOTS_A5, "clock_mhz_for_peak": f_peak,
+                    "gaussians_per_s": float(K) * T * d_out / (ms / 1e3),
+                    "gemm_tflops": 2.0 * T * d_in * d_out / (ms / 1e3) / 1e12,
+                    "peak_source": "148 SMs x 4 schedulers x 32 lanes x max SM clock"}
         elif kind in ("weight_grad", "logits"):
             fl = 2.0 * T * d_in * d_out
             ach = fl / (ms / 1e3) / 1e12

@@ -159,6 +159,33 @@ dust_status dust_layer_estimate_noalloc(const float *c, int T, int d_out,
                                         dust_noise nz, float *g_hat, void *g_hat_bf16,
                                         int accumulate, void *stream);
 
+/* ------------------------------------------------------------------ a1 + a5 + a6 fused
+ * [CA, error and weight equations] G_W[o][i] (+)= sum_t bf16(g_hat[t][o]) X[t][i]
+ * with g_hat as dust_layer_estimate computes it, produced tile by tile in
+ * shared memory as the tensor cores' operand and never written to device
+ * memory (unless g_hat_out is given): one kernel runs the draw reduction and
+ * the tcgen05 weight GEMM, with the d_in-wide row block of G_W held in TMEM.
+ *   c_or_r, is_r, T, d_out, seq_offsets, n_seq, gamma, nz: as
+ *     dust_layer_estimate (the reward scan, when needed, runs first into the
+ *     workspace);
+ *   X: [T][d_in] bf16, 16-byte aligned; d_in a multiple of 64, at most 512
+ *     (one CTA's TMEM holds 512 fp32 columns), else DUST_ERR_UNSUPPORTED;
+ *   G_W: [d_out][d_in] fp32, overwritten (accumulate = 0) or added to;
+ *   g_hat_out: nullable [T][d_out] fp32, receives g_hat (the same bits as
+ *     dust_layer_estimate's g_hat) for checks.
+ * The bf16 g values are those of dust_layer_estimate's g_hat_bf16, so G_W
+ * agrees with dust_layer_estimate followed by dust_weight_grad up to the
+ * order of the fp32 accumulation.  Token splits are summed in a fixed order.
+ * Workspace: dust_layer_estimate_weight_grad_workspace(); its first 256 bytes
+ * are the status block read by dust_poll_status. */
+dust_status dust_layer_estimate_weight_grad(const float *c_or_r, int is_r, int T, int d_out,
+                                            const int32_t *seq_offsets, int n_seq, float gamma,
+                                            dust_noise nz, const void *X, int d_in, float *G_W,
+                                            int accumulate, float *g_hat_out, void *ws, size_t ws_bytes,
+                                            void *stream);
+size_t dust_layer_estimate_weight_grad_workspace(int draw_count, int T, int d_in, int d_out, int is_r,
+                                                 float gamma);
+
 /* ------------------------------------------------------------------ a6: weight
  * [CA, weight equation] G_W[o][i] (+)= sum_t g_hat[t][o] X[t][i].
  * g_hat: [T][d_out], X: [T][d_in], both of dtype `dt` (DUST_BF16 runs on the

@@ -119,6 +119,24 @@ def test_workspace_queries_are_consistent(L):
     assert L.dust_head_step_workspace(64, 32, 512, 1, 1, 0) < L.dust_head_step_workspace(64, 32, 512, 1, 0, 0)
 
 
+def test_fused_estimate_rejected_on_host(L):
+    """dust_layer_estimate_weight_grad: d_in outside {64, ..., 512} step 64 is
+    unsupported, bad sizes / pointers / workspaces are rejected before launch."""
+    st = None
+    f = L.dust_layer_estimate_weight_grad
+    need = L.dust_layer_estimate_weight_grad_workspace(4, 96, 128, 40, 1, 0.0)
+    assert need > 256
+    assert L.dust_layer_estimate_weight_grad_workspace(4, 96, 1024, 40, 1, 0.0) == 256      # unsupported d_in
+    for d_in in (1024, 100, 0, 32):
+        assert status(f(GOOD, 1, 96, 40, None, 1, 0.0, NZ.c(), GOOD, d_in, GOOD, 0, None, GOOD, 1 << 30, st)) == 2
+    assert status(f(GOOD, 1, 0, 40, None, 1, 0.0, NZ.c(), GOOD, 128, GOOD, 0, None, GOOD, 1 << 30, st)) == 1
+    assert status(f(GOOD, 1, 96, 40, None, 1, 0.0, NZ.c(), GOOD + 8, 128, GOOD, 0, None, GOOD, 1 << 30, st)) == 3
+    assert status(f(GOOD, 1, 96, 40, None, 1, 0.0, NZ.c(), GOOD, 128, None, 0, None, GOOD, 1 << 30, st)) == 1
+    assert status(f(GOOD, 1, 96, 40, None, 1, 0.0, NZ.c(), GOOD, 128, GOOD, 0, None, GOOD, need - 1, st)) == 4
+    need_scan = L.dust_layer_estimate_weight_grad_workspace(4, 96, 128, 40, 0, 0.9)
+    assert need_scan >= need + 4 * 96 * 4
+
+
 def test_binding_rejects_host_tensors():
     import torch
     with pytest.raises(ValueError):

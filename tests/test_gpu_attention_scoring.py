@@ -8,6 +8,8 @@ import torch
 from activation_perturbation_es_b200 import dust
 from activation_perturbation_es_b200 import inputs as I
 
+import oracle_chains  # noqa: E402
+
 pytestmark = pytest.mark.gpu
 
 
@@ -46,20 +48,26 @@ def test_attention_costs_parity(orc, which):
 
 
 def test_value_projection_estimate_end_to_end(orc):
+    """The value projection's costs for every draw against the oracle's, then
+    the estimator and the weight estimate on the oracle's costs."""
     p = _block(seed=51)
     K, dh = 48, 64
     nz = dust.Noise(4, 22, 0, K, K, 0.01)
     goff = cu(p["off"])
     c = dust.attention_internal_costs(cu(p["Y"]), goff, cu(p["Wq"]), cu(p["Wk"]), cu(p["Wv"]), cu(p["Wo"]), 2,
                                       cu(p["G"]), nz)
-    g, _ = dust.layer_estimate(c, False, goff, 1.0, nz, dh)
+    c_orc = orc.attention_internal_costs(p["Y"], p["off"], p["Wq"], p["Wk"], p["Wv"], p["Wo"], 2, p["G"], 4, 22,
+                                         0.01, np.arange(K)).astype(np.float32)
+    assert rel_err(c.cpu().numpy(), c_orc) < 1e-3
+    g, _ = dust.layer_estimate(cu(c_orc), False, goff, 1.0, nz, dh)
     G_W = dust.weight_grad(g, cu(p["Y"]))                  # the value projection's input is Y
     toks = np.array([0, 255, 256, 1023])
-    c_h = c.cpu().numpy()
-    g_ref = orc.layer_estimate(c_h, False, dh, p["off"], 1.0, 4, 22, 0, K, 0.01, toks)
+    g_ref = orc.layer_estimate(c_orc, False, dh, p["off"], 1.0, 4, 22, 0, K, 0.01, toks)
     assert rel_err(g.cpu().numpy()[toks], g_ref) < 1e-3
     rows = np.array([0, 63])
-    assert rel_err(G_W.cpu().numpy()[rows], orc.weight_grad(g.cpu().numpy(), p["Y"], rows=rows)) < 1e-5
+    G_ref = oracle_chains.weight_rows(orc, c_orc, False, dh, p["off"], 1.0, 4, 22, 0, K, 0.01, p["Y"], rows,
+                                      bf16=False)
+    assert rel_err(G_W.cpu().numpy()[rows], G_ref) < 1e-4
 
 
 def test_value_estimate_converges_through_uniform_attention():

@@ -32,9 +32,10 @@ def _head(T=512, d=64, V=512, seed=0):
 def test_head_bp_grad_parity(orc, dt):
     X, W, y = _head(T=700, d=48, V=384)
     Xg = torch.from_numpy(X).cuda().to(dt)
-    Z = dust.logits(Xg, torch.from_numpy(W).cuda().to(dt))
-    G = dust.head_bp_grad(Z, torch.from_numpy(y).cuda(), Xg).cpu().numpy()
-    ref = orc.head_bp_grad(Z.cpu().numpy(), y, X)
+    # both sides get the oracle's logits (binary32); the logits GEMM is pinned on its own
+    Z = orc.logits(X, W).astype(np.float32)
+    G = dust.head_bp_grad(torch.from_numpy(Z).cuda(), torch.from_numpy(y).cuda(), Xg).cpu().numpy()
+    ref = orc.head_bp_grad(Z, y, X)
     # bf16: the softmax difference is rounded to bf16 before the tensor-core GEMM
     assert rel_err(G, ref) < (2e-2 if dt == torch.bfloat16 else 1e-5)
 
