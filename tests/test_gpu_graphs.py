@@ -35,6 +35,7 @@ def test_step_replays_from_a_cuda_graph():
     gh = torch.empty(T, V, device="cuda")
     gh16 = torch.empty(T, V, device="cuda", dtype=torch.bfloat16)
     GH = torch.empty(V, d_in, device="cuda")
+    GF = torch.empty(d_out, d_in, device="cuda")
     stream = torch.cuda.Stream()
 
     def step():
@@ -44,17 +45,18 @@ def test_step_replays_from_a_cuda_graph():
         dust.logits(X, W, Z=Z)
         dust.head_step(y, Vc, nz_h, Z=Z, g_hat=gh, g_hat_bf16=gh16)
         dust.weight_grad(gh16, X, G_W=GH)
+        dust.layer_estimate_weight_grad(r, True, off, 0.9, nz_l, X, d_out, G_W=GF)   # fused a5 + a6
 
     with torch.cuda.stream(stream):
         step()                                   # warm-up: workspaces, kernel attributes
     torch.cuda.synchronize()
-    eager = [t.clone() for t in (g, G, gh, GH)]
-    for t in (g, G, gh, GH):
+    eager = [t.clone() for t in (g, G, gh, GH, GF)]
+    for t in (g, G, gh, GH, GF):
         t.zero_()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         step()
     graph.replay()
     torch.cuda.synchronize()
-    for a, b in zip(eager, (g, G, gh, GH)):
+    for a, b in zip(eager, (g, G, gh, GH, GF)):
         assert torch.equal(a, b)
