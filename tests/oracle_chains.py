@@ -3,8 +3,7 @@ checks whose reference needs a whole column of the error estimate: every
 oracle input here comes from the seeded generators or from other oracle
 calls, never from the GPU."""
 import numpy as np
-
-from activation_perturbation_es_b200 import inputs as I
+import torch
 
 
 def weight_rows(orc, c_or_r, is_r, d_out, offsets, gamma, seed, layer, draw_begin, K_total, sigma, X, rows,
@@ -23,5 +22,6 @@ def weight_rows(orc, c_or_r, is_r, d_out, offsets, gamma, seed, layer, draw_begi
     g = orc.layer_estimate(c_or_r, True, d_out, offsets, gamma, seed, layer, draw_begin, K_total, sigma,
                            np.arange(T), chans=rows).astype(np.float32)
     if bf16:
-        g = I.bf16_round(g)
+        # round to nearest bf16, ties to even (torch's CPU conversion)
+        g = torch.from_numpy(g).to(torch.bfloat16).float().numpy()
     return orc.weight_grad(g, X, rows=np.arange(len(rows)))
