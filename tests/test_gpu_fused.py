@@ -113,3 +113,29 @@ def test_fused_rejects_unsupported_width():
         with pytest.raises(dust.DustError) as e:
             dust.layer_estimate_weight_grad(c, True, None, 0.0, nz, X, 32)
         assert e.value.status == 2
+
+
+@pytest.mark.parametrize("split", [1, 3, 5])
+def test_fused_draw_ranges_add_up(orc, split):
+    """Draw sharding (each call a range of the draws, all scaled by K_total):
+    the fused calls added with accumulate = 1 give the one-call G_W up to the
+    fp32 order of the sums."""
+    T, d_out, d_in, K, gamma = 400, 160, 256, 8, 0.9
+    off_h = I.offsets_from_lengths(I.ragged_lengths(T, 3, seed=4))
+    off = cu(off_h)
+    c = I.normal((K, T), 0.02, seed=6)
+    X_h = I.bf16_round(I.normal((T, d_in), 1.0, seed=7))
+    X = cu(X_h, torch.bfloat16)
+    G_all, _ = dust.layer_estimate_weight_grad(cu(c), False, off, gamma, dust.Noise(1, 2, 0, K, K, 0.01), X, d_out)
+    G = torch.zeros(d_out, d_in, device="cuda")
+    dust.layer_estimate_weight_grad(cu(c[:split]), False, off, gamma, dust.Noise(1, 2, 0, split, K, 0.01), X, d_out,
+                                    G_W=G, accumulate=True)
+    dust.layer_estimate_weight_grad(cu(c[split:]), False, off, gamma, dust.Noise(1, 2, split, K - split, K, 0.01), X,
+                                    d_out, G_W=G, accumulate=True)
+    # each call rounds its own partial g to bf16: the oracle chain does the same per range
+    rows = np.arange(d_out)
+    G_ref = (oracle_chains.weight_rows(orc, c[:split], False, d_out, off_h, gamma, 1, 2, 0, K, 0.01, X_h, rows) +
+             oracle_chains.weight_rows(orc, c[split:], False, d_out, off_h, gamma, 1, 2, split, K, 0.01, X_h, rows))
+    assert rel_err(host(G), G_ref) < BF16_G_TOL
+    # and against the one-call estimate at bf16 resolution (the roundings differ)
+    assert rel_err(host(G), host(G_all).astype(np.float64)) < 2e-2

@@ -77,7 +77,7 @@ def test_head_random_shapes(orc, T, n_chunks, Vc, K, sigma, seed):
 
 
 @settings(**dict(SETTINGS, max_examples=30))
-@given(lengths=lengths_st, d_out=st.integers(1, 300), d_in=st.sampled_from([64, 128, 192, 320, 512]),
+@given(lengths=lengths_st, d_out=st.integers(1, 300), d_in=st.sampled_from([64, 128, 192, 256, 320, 384, 448, 512]),
        K=st.integers(1, 7), gamma=gamma_st, seed=st.integers(0, 10_000))
 def test_fused_random_shapes(orc, lengths, d_out, d_in, K, gamma, seed):
     """Fused reduction + weight estimate against the oracle's chain."""
