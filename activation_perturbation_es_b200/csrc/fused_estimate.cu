@@ -18,7 +18,7 @@
 //     MN-major, 128-byte-swizzled layout that TMA would have produced; then a
 //     proxy fence and one arrive per warp on the stage's a_full barrier;
 //   warp 0, one lane: TMA loads of the stage's X tile (d_in/64 atoms of kTs
-//     rows, no multicast) onto x_full;
+//     rows, into this CTA only) onto x_full;
 //   warp 1, one lane: allocates TMEM, and per stage issues kTs/16 K steps of
 //     tcgen05.mma (M = 128, N <= 256 per instruction) and commits the stage's
 //     empty barrier.

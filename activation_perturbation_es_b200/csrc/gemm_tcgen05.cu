@@ -11,7 +11,7 @@
 // Tile 128 x BN (BN in {64, 128, 256}), 64-deep k blocks in a 4-stage ring.
 // One CTA of 4 warps per output tile and k slice:
 //   warp 0, one lane: TMA producer (cp.async.bulk.tensor, 128-byte swizzle,
-//           no multicast), one mbarrier per stage with expected bytes;
+//           each CTA loads its own tiles), one mbarrier per stage with expected bytes;
 //   warp 1, one lane: MMA issuer, 4 x tcgen05.mma (M = 128, N = BN, K = 16)
 //           per stage, tcgen05.commit frees the stage; warp 1 also allocates
 //           and frees the TMEM accumulator (BN fp32 columns);

@@ -1,5 +1,5 @@
 // tcgen05.cuh -- PTX wrappers for the sm_100a tensor-core kernels: mbarriers
-// with bounded waits, 2-D TMA loads (no multicast), TMEM allocation, tcgen05
+// with bounded waits, 2-D TMA loads into the issuing CTA, TMEM allocation, tcgen05
 // MMA / commit / load, and the shared-memory matrix descriptor.
 #pragma once
 #include <cuda.h>
