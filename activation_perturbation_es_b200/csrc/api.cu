@@ -50,6 +50,7 @@ dust_status check_noise(const dust_noise& nz) {
     DUST_REQUIRE(std::isfinite(nz.sigma) && nz.sigma > 0.0f, DUST_ERR_INVALID_ARG, "sigma must be finite and > 0");
     DUST_REQUIRE(static_cast<uint64_t>(nz.draw_begin) + nz.draw_count <= (1ull << 32), DUST_ERR_INVALID_ARG,
                  "draw_begin + draw_count exceeds 2^32");
+    DUST_REQUIRE(nz.token_begin <= 0x7FFFFFFFu, DUST_ERR_INVALID_ARG, "token_begin must be < 2^31");
     return ok();
 }
 
@@ -285,6 +286,9 @@ dust_status dust_layer_estimate_weight_grad(const float* c_or_r, int is_r, int T
                  "gamma must be in [0, 1]");
     DUST_REQUIRE(static_cast<long long>(nz.draw_count) * T < (1ll << 31), DUST_ERR_INVALID_ARG,
                  "draw_count x T must be < 2^31");
+    DUST_REQUIRE(nz.draw_count <= dust::kFusedMaxDraws, DUST_ERR_UNSUPPORTED,
+                 "draw_count must be <= %u per call (split the draws over calls with accumulate = 1)",
+                 dust::kFusedMaxDraws);
     DUST_TRY(check_ptr(c_or_r, "c_or_r"));
     DUST_TRY(check_ptr(X, "X"));
     DUST_TRY(check_ptr(G_W, "G_W"));
@@ -317,26 +321,39 @@ static GemmPlan weight_grad_plan(int T, int d_in, int d_out, dust_dtype dt) {
     return plan_gemm(d_out, d_in, T, dt, false, false);
 }
 
-size_t dust_weight_grad_workspace(int T, int d_in, int d_out, dust_dtype dt) {
+// Operands of one type take that type's GEMM (bf16: tcgen05 where the shape
+// allows); mixed types take the CUDA-core GEMM with both widened to fp32.
+static GemmPlan weight_grad_plan2(int T, int d_in, int d_out, dust_dtype g_dt, dust_dtype x_dt) {
+    return g_dt == x_dt ? weight_grad_plan(T, d_in, d_out, g_dt) : plan_gemm(d_out, d_in, T, DUST_F32, false, false);
+}
+
+size_t dust_weight_grad_workspace(int T, int d_in, int d_out, dust_dtype g_dt, dust_dtype x_dt) {
     Layout L;
-    if (T > 0 && d_in > 0 && d_out > 0) L.add(weight_grad_plan(T, d_in, d_out, dt).partial_bytes);
+    if (T > 0 && d_in > 0 && d_out > 0) L.add(weight_grad_plan2(T, d_in, d_out, g_dt, x_dt).partial_bytes);
     return L.off;
 }
 
-dust_status dust_weight_grad(const void* g_hat, const void* X, dust_dtype dt, int T, int d_in, int d_out,
-                             float* G_W, int accumulate, void* ws, size_t ws_bytes, void* stream) {
-    DUST_REQUIRE(dt == DUST_F32 || dt == DUST_BF16, DUST_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
+dust_status dust_weight_grad(const void* g_hat, dust_dtype g_dt, const void* X, dust_dtype x_dt, int T, int d_in,
+                             int d_out, float* G_W, int accumulate, void* ws, size_t ws_bytes, void* stream) {
+    DUST_REQUIRE(g_dt == DUST_F32 || g_dt == DUST_BF16, DUST_ERR_INVALID_ARG, "unknown g dtype %d",
+                 static_cast<int>(g_dt));
+    DUST_REQUIRE(x_dt == DUST_F32 || x_dt == DUST_BF16, DUST_ERR_INVALID_ARG, "unknown X dtype %d",
+                 static_cast<int>(x_dt));
     DUST_REQUIRE(T > 0 && d_in > 0 && d_out > 0, DUST_ERR_INVALID_ARG, "T, d_in, d_out must be > 0");
     DUST_TRY(check_ptr(g_hat, "g_hat"));
     DUST_TRY(check_ptr(X, "X"));
     DUST_TRY(check_ptr(G_W, "G_W"));
     DUST_TRY(check_ptr(ws, "ws"));
-    const size_t need = dust_weight_grad_workspace(T, d_in, d_out, dt);
+    const size_t need = dust_weight_grad_workspace(T, d_in, d_out, g_dt, x_dt);
     DUST_REQUIRE(ws_bytes >= need, DUST_ERR_WORKSPACE, "workspace %zu bytes < %zu", ws_bytes, need);
-    const GemmPlan p = weight_grad_plan(T, d_in, d_out, dt);
+    const GemmPlan p = weight_grad_plan2(T, d_in, d_out, g_dt, x_dt);
     float* partial = reinterpret_cast<float*>(region(ws, dust::kStatusBytes));
-    return run_gemm(p, g_hat, false, d_out, X, false, d_in, dt, d_out, d_in, T, G_W, d_in, accumulate, partial,
-                    static_cast<uint32_t*>(ws), as_stream(stream));
+    if (g_dt == x_dt)
+        return run_gemm(p, g_hat, false, d_out, X, false, d_in, g_dt, d_out, d_in, T, G_W, d_in, accumulate, partial,
+                        static_cast<uint32_t*>(ws), as_stream(stream));
+    return cuda_status(dust::launch_gemm_simt_mixed(g_hat, g_dt, false, d_out, X, x_dt, false, d_in, d_out, d_in, T,
+                                                    G_W, d_in, accumulate, partial, p.splits, as_stream(stream)),
+                       "CUDA-core GEMM (mixed operand types)");
 }
 
 // ------------------------------------------------------------------ a2
@@ -384,7 +401,9 @@ struct HeadLayout {
     GemmPlan zplan, wplan;
 };
 
-HeadLayout head_layout(int T, int d_in, int V, dust_dtype dt, int has_Z, int want_G_W) {
+// Vr = the call's vocabulary range (chunk_count x Vc): g and its bf16 copy are
+// [T][Vr], G_W [Vr][d_in]; the logits and their statistics cover all V.
+HeadLayout head_layout(int T, int d_in, int V, int Vr, dust_dtype dt, int has_Z, int want_G_W) {
     HeadLayout h;
     Layout L;
     if (!has_Z) {
@@ -394,8 +413,8 @@ HeadLayout head_layout(int T, int d_in, int V, dust_dtype dt, int has_Z, int wan
     }
     h.lse = L.add(sizeof(float) * static_cast<size_t>(T));
     if (want_G_W) {
-        h.wplan = weight_grad_plan(T, d_in, V, dt);
-        if (dt == DUST_BF16) h.g16 = L.add(sizeof(uint16_t) * static_cast<size_t>(T) * V);
+        h.wplan = weight_grad_plan(T, d_in, Vr, dt);
+        if (dt == DUST_BF16) h.g16 = L.add(sizeof(uint16_t) * static_cast<size_t>(T) * Vr);
         h.wpart = L.add(h.wplan.partial_bytes);
     }
     h.total = L.off;
@@ -403,14 +422,17 @@ HeadLayout head_layout(int T, int d_in, int V, dust_dtype dt, int has_Z, int wan
 }
 }  // namespace
 
-size_t dust_head_step_workspace(int T, int d_in, int V, dust_dtype dt, int has_Z, int want_G_W) {
-    if (T <= 0 || V <= 0 || ((!has_Z || want_G_W) && d_in <= 0)) return dust::kStatusBytes;
-    return head_layout(T, d_in, V, dt, has_Z, want_G_W).total;
+size_t dust_head_step_workspace(int T, int d_in, int V, int Vc, int chunk_count, dust_dtype dt, int has_Z,
+                                int want_G_W) {
+    if (T <= 0 || V <= 0 || Vc <= 0 || chunk_count <= 0 || ((!has_Z || want_G_W) && d_in <= 0))
+        return dust::kStatusBytes;
+    return head_layout(T, d_in, V, Vc * chunk_count, dt, has_Z, want_G_W).total;
 }
 
 dust_status dust_head_step(const void* X, const void* W, dust_dtype dt, const float* Z, const int32_t* targets, int T,
-                           int d_in, int V, int Vc, dust_noise nz, float* c_out, float* g_hat, void* g_hat_bf16,
-                           float* G_W, int accumulate, void* ws, size_t ws_bytes, void* stream) {
+                           int d_in, int V, int Vc, int chunk_begin, int chunk_count, dust_noise nz, float* c_out,
+                           float* g_hat, void* g_hat_bf16, float* G_W, int accumulate, void* ws, size_t ws_bytes,
+                           void* stream) {
     DUST_TRY(check_noise(nz));
     DUST_REQUIRE(dt == DUST_F32 || dt == DUST_BF16, DUST_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
     DUST_REQUIRE(T > 0 && V > 0, DUST_ERR_INVALID_ARG, "T and V must be > 0");
@@ -418,6 +440,9 @@ dust_status dust_head_step(const void* X, const void* W, dust_dtype dt, const fl
     DUST_REQUIRE(dust::head_chunk_supported(Vc), DUST_ERR_UNSUPPORTED,
                  "Vc=%d unsupported (multiples of 128 up to 1024, of 256 up to 2048, of 512 up to 4096)", Vc);
     DUST_REQUIRE(V / Vc <= 65535, DUST_ERR_INVALID_ARG, "too many chunks");
+    DUST_REQUIRE(chunk_begin >= 0 && chunk_count > 0 && chunk_begin + chunk_count <= V / Vc, DUST_ERR_INVALID_ARG,
+                 "chunk range [%d, %d) outside the %d chunks", chunk_begin, chunk_begin + chunk_count, V / Vc);
+    const int Vr = chunk_count * Vc;
     const bool has_Z = Z != nullptr, want_G_W = G_W != nullptr;
     if (!has_Z || want_G_W) {
         DUST_REQUIRE(d_in > 0, DUST_ERR_INVALID_ARG, "d_in must be > 0");
@@ -431,7 +456,7 @@ dust_status dust_head_step(const void* X, const void* W, dust_dtype dt, const fl
     DUST_TRY(check_ptr(g_hat_bf16, "g_hat_bf16", true));
     DUST_TRY(check_ptr(G_W, "G_W", true));
     DUST_TRY(check_ptr(ws, "ws"));
-    const HeadLayout h = head_layout(T, d_in, V, dt, has_Z, want_G_W);
+    const HeadLayout h = head_layout(T, d_in, V, Vr, dt, has_Z, want_G_W);
     DUST_REQUIRE(ws_bytes >= h.total, DUST_ERR_WORKSPACE, "workspace %zu bytes < %zu", ws_bytes, h.total);
     cudaStream_t st = as_stream(stream);
     uint32_t* status = static_cast<uint32_t*>(ws);
@@ -447,11 +472,12 @@ dust_status dust_head_step(const void* X, const void* W, dust_dtype dt, const fl
     DUST_TRY(cuda_status(dust::launch_row_stats(Zuse, targets, T, V, lse, nullptr, st), "dust_head_step (row stats)"));
     void* g16 = g_hat_bf16;
     if (want_G_W && dt == DUST_BF16 && g16 == nullptr) g16 = region(ws, h.g16);
-    DUST_TRY(cuda_status(dust::launch_head_chunks(Zuse, lse, targets, T, V, Vc, nz, c_out, g_hat, g16, accumulate, st),
+    DUST_TRY(cuda_status(dust::launch_head_chunks(Zuse, lse, targets, T, V, Vc, chunk_begin, chunk_count, nz, c_out,
+                                                  g_hat, g16, accumulate, st),
                          "dust_head_step (chunks)"));
     if (!want_G_W) return ok();
     const void* gA = dt == DUST_BF16 ? g16 : static_cast<const void*>(g_hat);
-    return run_gemm(h.wplan, gA, false, V, X, false, d_in, dt, V, d_in, T, G_W, d_in, 0,
+    return run_gemm(h.wplan, gA, false, Vr, X, false, d_in, dt, Vr, d_in, T, G_W, d_in, 0,
                     reinterpret_cast<float*>(region(ws, h.wpart)), status, st);
 }
 
@@ -521,6 +547,8 @@ dust_status dust_noise_fill(dust_noise nz, uint32_t stream_id, int t0, int n_tok
                             void* stream) {
     DUST_REQUIRE(nz.draw_count > 0, DUST_ERR_INVALID_ARG, "draw_count must be > 0");
     DUST_REQUIRE(t0 >= 0 && n_tok > 0 && j0 >= 0 && n_ch > 0, DUST_ERR_INVALID_ARG, "bad token/channel range");
+    DUST_REQUIRE(static_cast<uint64_t>(nz.token_begin) + static_cast<uint64_t>(t0) + n_tok <= (1ull << 32),
+                 DUST_ERR_INVALID_ARG, "token_begin + t0 + n_tok exceeds 2^32");
     DUST_TRY(check_ptr(out, "out"));
     return cuda_status(dust::launch_noise_fill(nz, stream_id, t0, n_tok, j0, n_ch, out, as_stream(stream)),
                        "dust_noise_fill");
@@ -542,6 +570,7 @@ dust_status dust_synth_costs(const float* u, int T, int d_out, dust_noise nz, fl
     DUST_REQUIRE(std::isfinite(eps_scale), DUST_ERR_INVALID_ARG, "eps_scale must be finite");
     DUST_REQUIRE(T > 0 && d_out > 0, DUST_ERR_INVALID_ARG, "T and d_out must be > 0");
     DUST_REQUIRE(nz.draw_count <= 65535u * 32u, DUST_ERR_INVALID_ARG, "draw_count must be <= 2097120");
+    DUST_REQUIRE(nz.token_begin <= 0x7FFFFFFFu, DUST_ERR_INVALID_ARG, "token_begin must be < 2^31");
     DUST_TRY(check_ptr(u, "u"));
     DUST_TRY(check_ptr(c, "c"));
     return cuda_status(dust::launch_synth_costs(u, T, d_out, nz, eps_scale, c, as_stream(stream)), "dust_synth_costs");
@@ -578,12 +607,18 @@ size_t dust_attention_internal_costs_workspace(int draw_count, int T, int d, int
 }
 
 dust_status dust_attention_internal_costs(const float* Y, int T, int d, const int32_t* seq_offsets, int n_seq,
-                                          const float* Wq, const float* Wk, const float* Wv, const float* Wo, int dh,
-                                          int which, const float* G, dust_noise nz, float* c, void* ws,
-                                          size_t ws_bytes, void* stream) {
+                                          const float* Wq, const float* Wk, const float* Wv, const float* Wo,
+                                          const float* Wg, const float* E, int dh, int which, const float* G,
+                                          dust_noise nz, float* c, void* ws, size_t ws_bytes, void* stream) {
     DUST_TRY(check_noise(nz));
     DUST_REQUIRE(T > 0 && d > 0 && dh > 0, DUST_ERR_INVALID_ARG, "T, d, dh must be > 0");
-    DUST_REQUIRE(which >= 0 && which <= 2, DUST_ERR_INVALID_ARG, "which must be 0 (q), 1 (k) or 2 (v)");
+    DUST_REQUIRE(which >= 0 && which <= 4, DUST_ERR_INVALID_ARG,
+                 "which must be 0 (q), 1 (k), 2 (v), 3 (gate) or 4 (value embedding)");
+    DUST_REQUIRE(which != 3 || (Wg != nullptr && E != nullptr), DUST_ERR_INVALID_ARG,
+                 "gate draws need the gate's weights Wg and the value embeddings E");
+    DUST_REQUIRE(which != 4 || E != nullptr, DUST_ERR_INVALID_ARG, "value-embedding draws need E");
+    DUST_TRY(check_ptr(Wg, "Wg", true));
+    DUST_TRY(check_ptr(E, "E", true));
     DUST_REQUIRE(dh % 4 == 0 && dh <= 128, DUST_ERR_UNSUPPORTED, "attention scoring supports dh %% 4 == 0, dh <= 128");
     DUST_TRY(check_seq(seq_offsets, n_seq, 1, T));
     const void* ptrs[] = {Y, Wq, Wk, Wv, Wo, G, c, ws};
@@ -591,8 +626,8 @@ dust_status dust_attention_internal_costs(const float* Y, int T, int d, const in
     for (int i = 0; i < 8; ++i) DUST_TRY(check_ptr(ptrs[i], names[i]));
     const size_t need = dust_attention_internal_costs_workspace(static_cast<int>(nz.draw_count), T, d, dh);
     DUST_REQUIRE(ws_bytes >= need, DUST_ERR_WORKSPACE, "workspace %zu bytes < %zu", ws_bytes, need);
-    return cuda_status(dust::run_attention_internal_costs(Y, T, d, seq_offsets, n_seq, Wq, Wk, Wv, Wo, dh, which, G,
-                                                          nz, c, ws, as_stream(stream)),
+    return cuda_status(dust::run_attention_internal_costs(Y, T, d, seq_offsets, n_seq, Wq, Wk, Wv, Wo, Wg, E, dh,
+                                                          which, G, nz, c, ws, as_stream(stream)),
                        "dust_attention_internal_costs");
 }
 

@@ -21,9 +21,10 @@ namespace dust {
 
 namespace {
 
-// out[b][t][e] = P[t][e] + sigma a(first_draw + b, t, e)
+// out[b][t][e] = P[t][e] + sigma a(first_draw + b, tok0 + t, e)
 __global__ void perturb_projection_kernel(const float* __restrict__ P, int T, int dh, uint32_t seed, uint32_t layer,
-                                          uint32_t first_draw, int nb, float sigma, float* __restrict__ out) {
+                                          uint32_t tok0, uint32_t first_draw, int nb, float sigma,
+                                          float* __restrict__ out) {
     const int nq = dh / 4;
     const long long total = static_cast<long long>(nb) * T * nq;
     for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
@@ -33,13 +34,61 @@ __global__ void perturb_projection_kernel(const float* __restrict__ P, int T, in
         const int t = static_cast<int>(rest % T);
         const int b = static_cast<int>(rest / T);
         float4 p = __ldg(reinterpret_cast<const float4*>(P + static_cast<size_t>(t) * dh) + q);
-        const float4 a = gauss4(seed, layer, first_draw + static_cast<uint32_t>(b), static_cast<uint32_t>(t),
+        const float4 a = gauss4(seed, layer, first_draw + static_cast<uint32_t>(b), tok0 + static_cast<uint32_t>(t),
                                 static_cast<uint32_t>(q), 0);
         p.x = fmaf(sigma, a.x, p.x);
         p.y = fmaf(sigma, a.y, p.y);
         p.z = fmaf(sigma, a.z, p.z);
         p.w = fmaf(sigma, a.w, p.w);
         reinterpret_cast<float4*>(out + static_cast<size_t>(b * static_cast<long long>(T) + t) * dh)[q] = p;
+    }
+}
+
+__device__ __forceinline__ float logistic(float x) { return 1.0f / (1.0f + expf(-x)); }
+
+// v[t][e] += s(gp[t][e]) E[t][e] (s = 1 without a gate): the clean values carry
+// the token's gated value embedding
+__global__ void gated_values_kernel(float* __restrict__ v, const float* __restrict__ gp,
+                                    const float* __restrict__ E, long long n) {
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x)
+        v[i] = fmaf(gp ? logistic(__ldg(gp + i)) : 1.0f, __ldg(E + i), v[i]);
+}
+
+// The perturbed values of a draw batch when the gate's pre-activation (GATE)
+// or the value embedding (else) takes the noise h = sigma a(first_draw + b, tok0 + t, e):
+//   gate:  v~ = v + (s(g + h) - s(g)) E, the difference formed without
+//          cancellation as (1 - s(g)) s(g + h) (-expm1(-h));
+//   value embedding: v~ = v + s(g) h (s = 1 without a gate).
+template <bool GATE>
+__global__ void perturb_values_kernel(const float* __restrict__ v, const float* __restrict__ gp,
+                                      const float* __restrict__ E, int T, int dh, uint32_t seed, uint32_t layer,
+                                      uint32_t tok0, uint32_t first_draw, int nb, float sigma,
+                                      float* __restrict__ out) {
+    const int nq = dh / 4;
+    const long long total = static_cast<long long>(nb) * T * nq;
+    for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
+         idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int q = static_cast<int>(idx % nq);
+        const long long rest = idx / nq;
+        const int t = static_cast<int>(rest % T);
+        const int b = static_cast<int>(rest / T);
+        const size_t i0 = static_cast<size_t>(t) * dh + 4 * q;
+        const float4 a = gauss4(seed, layer, first_draw + static_cast<uint32_t>(b), tok0 + static_cast<uint32_t>(t),
+                                static_cast<uint32_t>(q), 0);
+        const float av[4] = {a.x, a.y, a.z, a.w};
+        float o[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const float h = sigma * av[w];
+            const float g = gp ? __ldg(gp + i0 + w) : 0.0f;
+            float dv;
+            if (GATE) dv = (1.0f - logistic(g)) * logistic(g + h) * (-expm1f(-h)) * __ldg(E + i0 + w);
+            else dv = (gp ? logistic(g) : 1.0f) * h;
+            o[w] = __ldg(v + i0 + w) + dv;
+        }
+        reinterpret_cast<float4*>(out + static_cast<size_t>(b * static_cast<long long>(T) + t) * dh)[q] =
+            make_float4(o[0], o[1], o[2], o[3]);
     }
 }
 
@@ -65,7 +114,7 @@ unsigned grid_for(long long n) {
 }
 
 struct ScoreLayout {
-    size_t q, k, v, o, err, pp, op, part, total;
+    size_t q, k, v, gp, o, err, pp, op, part, total;
     int nb;
 };
 
@@ -78,6 +127,7 @@ ScoreLayout score_layout(int draw_count, int T, int d, int dh) {
     L.q = add(P);
     L.k = add(P);
     L.v = add(P);
+    L.gp = add(P);
     L.o = add(P);
     L.err = add(P);
     L.pp = add(P * L.nb);
@@ -100,14 +150,15 @@ size_t attention_scoring_workspace_bytes(int draw_count, int T, int d, int dh) {
 }
 
 cudaError_t run_attention_internal_costs(const float* Y, int T, int d, const int32_t* offs, int n_seq,
-                                         const float* Wq, const float* Wk, const float* Wv, const float* Wo, int dh,
-                                         int which, const float* G, const dust_noise& nz, float* c, void* ws,
-                                         cudaStream_t st) {
+                                         const float* Wq, const float* Wk, const float* Wv, const float* Wo,
+                                         const float* Wg, const float* E, int dh, int which, const float* G,
+                                         const dust_noise& nz, float* c, void* ws, cudaStream_t st) {
     const ScoreLayout L = score_layout(static_cast<int>(nz.draw_count), T, d, dh);
     auto* base = static_cast<uint8_t*>(ws);
     float* q = reinterpret_cast<float*>(base + L.q);
     float* k = reinterpret_cast<float*>(base + L.k);
     float* v = reinterpret_cast<float*>(base + L.v);
+    float* gp = Wg ? reinterpret_cast<float*>(base + L.gp) : nullptr;
     float* o = reinterpret_cast<float*>(base + L.o);
     float* err = reinterpret_cast<float*>(base + L.err);
     float* pp = reinterpret_cast<float*>(base + L.pp);
@@ -120,19 +171,37 @@ cudaError_t run_attention_internal_costs(const float* Y, int T, int d, const int
     for (int w = 0; w < 3 && e == cudaSuccess; ++w)
         e = launch_gemm_simt(Y, true, d, Ws[w], true, d, DUST_F32, T, dh, d, outs[w], dh, 0, part,
                              gemm_simt_splits(T, dh, d), st);
+    if (e == cudaSuccess && gp)      // the gate's pre-activation Y Wg^T
+        e = launch_gemm_simt(Y, true, d, Wg, true, d, DUST_F32, T, dh, d, gp, dh, 0, part,
+                             gemm_simt_splits(T, dh, d), st);
+    if (e == cudaSuccess && E) {
+        gated_values_kernel<<<grid_for(static_cast<long long>(T) * dh), 256, 0, st>>>(
+            v, gp, E, static_cast<long long>(T) * dh);
+        e = cudaGetLastError();
+    }
     if (e == cudaSuccess) e = launch_causal_attention(q, k, v, 0, 0, 0, 1, T, dh, offs, n_seq, o, st);
     if (e == cudaSuccess)   // err[t][e] = sum_j G[t][j] Wo[j][e]: B = Wo is [K = d][N = dh]
         e = launch_gemm_simt(G, true, d, Wo, false, dh, DUST_F32, T, dh, d, err, dh, 0, part,
                              gemm_simt_splits(T, dh, d), st);
     const float* P = which == 0 ? q : (which == 1 ? k : v);
     const long long bs = static_cast<long long>(T) * dh;
+    const bool on_v = which >= 2;    // v, the gate and the value embedding all act through the values
     for (int b0 = 0; b0 < static_cast<int>(nz.draw_count) && e == cudaSuccess; b0 += L.nb) {
         const int nb = std::min(L.nb, static_cast<int>(nz.draw_count) - b0);
-        perturb_projection_kernel<<<grid_for(static_cast<long long>(nb) * T * (dh / 4)), 256, 0, st>>>(
-            P, T, dh, nz.seed, nz.layer, nz.draw_begin + static_cast<uint32_t>(b0), nb, nz.sigma, pp);
+        const unsigned blocks = grid_for(static_cast<long long>(nb) * T * (dh / 4));
+        const uint32_t first = nz.draw_begin + static_cast<uint32_t>(b0);
+        if (which <= 2)
+            perturb_projection_kernel<<<blocks, 256, 0, st>>>(P, T, dh, nz.seed, nz.layer, nz.token_begin, first, nb,
+                                                              nz.sigma, pp);
+        else if (which == 3)
+            perturb_values_kernel<true><<<blocks, 256, 0, st>>>(v, gp, E, T, dh, nz.seed, nz.layer, nz.token_begin,
+                                                                first, nb, nz.sigma, pp);
+        else
+            perturb_values_kernel<false><<<blocks, 256, 0, st>>>(v, gp, E, T, dh, nz.seed, nz.layer, nz.token_begin,
+                                                                 first, nb, nz.sigma, pp);
         if ((e = cudaGetLastError()) != cudaSuccess) break;
-        e = launch_causal_attention(which == 0 ? pp : q, which == 1 ? pp : k, which == 2 ? pp : v,
-                                    which == 0 ? bs : 0, which == 1 ? bs : 0, which == 2 ? bs : 0, nb, T, dh, offs,
+        e = launch_causal_attention(which == 0 ? pp : q, which == 1 ? pp : k, on_v ? pp : v,
+                                    which == 0 ? bs : 0, which == 1 ? bs : 0, on_v ? bs : 0, nb, T, dh, offs,
                                     n_seq, op, st);
         if (e != cudaSuccess) break;
         const long long rows = static_cast<long long>(nb) * T;

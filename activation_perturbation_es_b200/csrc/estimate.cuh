@@ -24,4 +24,14 @@ __device__ __forceinline__ void accumulate_quad(float2& xz, float2& yw, float r,
     yw = __ffma2_rn(rr, p.sin_t, yw);
 }
 
+// accumulate_quad from the state after Philox round 1 (philox_round1_state).
+__device__ __forceinline__ void accumulate_quad_after_round1(float2& xz, float2& yw, float r, uint4 c1, uint32_t seed,
+                                                             uint32_t layer) {
+    const uint4 x = philox4x32_10_after_round1(c1, seed, layer);
+    const Polar2 p = box_muller_polar2(x.x, x.y, x.z, x.w);
+    const float2 rr = __fmul2_rn(splat(r), p.rho);
+    xz = __ffma2_rn(rr, p.cos_t, xz);
+    yw = __ffma2_rn(rr, p.sin_t, yw);
+}
+
 }  // namespace dust

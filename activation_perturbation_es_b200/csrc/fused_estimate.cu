@@ -45,9 +45,15 @@ constexpr int kRows = 128;                            // output channels per CTA
 constexpr int kAtom = kTs * 128;                      // one 64-wide MN atom of kTs K rows, bytes
 constexpr int kATile = 2 * kAtom;
 constexpr int kMaxStages = 4;
-// a stage's A tile fills only when the producers have run all K draws for
-// it, which at large K takes far longer than a pipeline hand-off
-constexpr uint32_t kProduceWaitLimit = 1u << 28;
+// A stage's A tile fills only when the producers have run all of the call's
+// draws for it, so the waits that span a stage's production are bounded in
+// time on the GPU's global nanosecond timer, by a budget that grows with the
+// draw count: 2 s plus 20 us per draw.  One draw of one stage is 48 tokens x
+// 128 channels of noise, about 1.2 us on one SM, so the budget is more than
+// ten times the longest legitimate wait.  The host caps a call at
+// kFusedMaxDraws draws (23 s).
+constexpr uint64_t kProduceBudgetBaseNs = 2000000000ull;
+constexpr uint64_t kProduceBudgetPerDrawNs = 20000ull;
 
 struct FusedLayout {
     int d_in, stage_bytes, stages, bytes;
@@ -73,6 +79,28 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     return false;
 }
 
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// The same wait, bounded by budget_ns of global-timer time (the poll count is
+// capped as well, as a last bound that does not depend on the timer).
+__device__ __forceinline__ bool wait_or_abort_ns(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                                 uint64_t budget_ns) {
+    const uint64_t start = global_ns();
+    for (uint32_t it = 0; it < 0xFFFFFFF0u; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (it > 64) {
+            __nanosleep(256);
+            if ((it & 255u) == 0u && global_ns() - start > budget_ns) return false;
+        }
+    }
+    return false;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -80,7 +108,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 
 __global__ void __launch_bounds__(kFusedThreads, 1)
 fused_estimate_kernel(const __grid_constant__ CUtensorMap map_x, const float* __restrict__ r, int T, int d_out,
-                      int d_in, uint32_t seed, uint32_t layer, uint32_t draw_begin, int nd, float scale,
+                      int d_in, uint32_t seed, uint32_t layer, uint32_t draw_begin, uint32_t tok0, int nd, float scale,
                       int tokens_per_split, float* __restrict__ partial, float* __restrict__ g_hat,
                       uint32_t* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
@@ -102,6 +130,7 @@ fused_estimate_kernel(const __grid_constant__ CUtensorMap map_x, const float* __
     const int te = min(T, tb + tokens_per_split);
     const int n_stages = te > tb ? (te - tb + kTs - 1) / kTs : 0;
     const uint32_t tmem_cols = d_in <= 64 ? 64u : (d_in <= 128 ? 128u : (d_in <= 256 ? 256u : 512u));
+    const uint64_t produce_limit = kProduceBudgetBaseNs + kProduceBudgetPerDrawNs * static_cast<uint64_t>(nd);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < L.stages; ++s) {
@@ -128,7 +157,7 @@ fused_estimate_kernel(const __grid_constant__ CUtensorMap map_x, const float* __
             for (; it < n_stages; ++it) {
                 const int s = it % L.stages;
                 if (it >= L.stages &&
-                    !wait_or_abort(&empty[s], ((it / L.stages) - 1) & 1, abort_flag, kProduceWaitLimit)) {
+                    !wait_or_abort_ns(&empty[s], ((it / L.stages) - 1) & 1, abort_flag, produce_limit)) {
                     ok = false;
                     break;
                 }
@@ -149,7 +178,7 @@ fused_estimate_kernel(const __grid_constant__ CUtensorMap map_x, const float* __
             bool ok = true;
             for (int it = 0; it < n_stages && ok; ++it) {
                 const int s = it % L.stages;
-                if (!wait_or_abort(&a_full[s], (it / L.stages) & 1, abort_flag, kProduceWaitLimit) ||
+                if (!wait_or_abort_ns(&a_full[s], (it / L.stages) & 1, abort_flag, produce_limit) ||
                     !wait_or_abort(&x_full[s], (it / L.stages) & 1, abort_flag, kWaitLimit)) {
                     ok = false;
                     break;
@@ -186,6 +215,7 @@ fused_estimate_kernel(const __grid_constant__ CUtensorMap map_x, const float* __
         // ---------------- producers: g tiles into shared memory
         const int pw = warp - 2;                    // 0 .. kProducerWarps - 1
         const uint32_t quad = static_cast<uint32_t>(o0 / 4 + lane);
+        const uint2 rq = philox_round1_quad(quad, 0u, layer);
         const int atom = lane >> 4;                 // channels 4q .. 4q+3 lie in MN atom q / 16
         const int chunk = (lane & 15) >> 1;         // 16-byte chunk of the 128-byte row
         const int half8 = (lane & 1) * 8;           // byte offset inside the chunk
@@ -193,7 +223,7 @@ fused_estimate_kernel(const __grid_constant__ CUtensorMap map_x, const float* __
         for (int it = 0; it < n_stages; ++it) {
             const int s = it % L.stages;
             if (it >= L.stages &&
-                !wait_or_abort(&empty[s], ((it / L.stages) - 1) & 1, abort_flag, kProduceWaitLimit)) {
+                !wait_or_abort_ns(&empty[s], ((it / L.stages) - 1) & 1, abort_flag, produce_limit)) {
                 ok = false;
                 break;
             }
@@ -203,30 +233,36 @@ fused_estimate_kernel(const __grid_constant__ CUtensorMap map_x, const float* __
             const bool v0 = t0 < te, v1 = t1 < te;      // warp-uniform
             float2 xa0 = splat(0.0f), ya0 = splat(0.0f), xa1 = splat(0.0f), ya1 = splat(0.0f);
             float2 xb0 = splat(0.0f), yb0 = splat(0.0f), xb1 = splat(0.0f), yb1 = splat(0.0f);
-            const float* ra = r + (v0 ? t0 : 0);
-            const float* rb = r + (v1 ? t1 : 0);
-            int k = 0;
-            if (v0 && v1) {
-                for (; k + 2 <= nd; k += 2) {
-                    const float a0 = __ldg(ra + static_cast<size_t>(k) * T), a1 = __ldg(ra + static_cast<size_t>(k + 1) * T);
-                    const float b0 = __ldg(rb + static_cast<size_t>(k) * T), b1 = __ldg(rb + static_cast<size_t>(k + 1) * T);
-                    accumulate_quad(xa0, ya0, a0, seed, layer, draw_begin + k, t0, quad);
-                    accumulate_quad(xb0, yb0, b0, seed, layer, draw_begin + k, t1, quad);
-                    accumulate_quad(xa1, ya1, a1, seed, layer, draw_begin + k + 1, t0, quad);
-                    accumulate_quad(xb1, yb1, b1, seed, layer, draw_begin + k + 1, t1, quad);
+            if (v0) {
+                // the standalone reduction's loop (same draw order and accumulator
+                // pairs) on two tokens; when t1 lies past the split it repeats t0
+                const int ta = t0, tb_ = v1 ? t1 : t0;
+                const float* ra = r + ta;
+                const float* rb = r + tb_;
+                const uint32_t ua = tok0 + static_cast<uint32_t>(ta), ub = tok0 + static_cast<uint32_t>(tb_);
+                DrawProduct dp = draw_product(draw_begin);
+                for (int k0 = 0; k0 < nd; k0 += 32) {
+                    const int n = nd - k0 < 32 ? nd - k0 : 32;
+                    const float rva = lane < n ? __ldg(ra + static_cast<size_t>(k0 + lane) * T) : 0.0f;
+                    const float rvb = lane < n ? __ldg(rb + static_cast<size_t>(k0 + lane) * T) : 0.0f;
+                    int j = 0;
+                    for (; j + 2 <= n; j += 2) {
+                        const float a0 = __shfl_sync(0xffffffffu, rva, j), a1 = __shfl_sync(0xffffffffu, rva, j + 1);
+                        const float b0 = __shfl_sync(0xffffffffu, rvb, j), b1 = __shfl_sync(0xffffffffu, rvb, j + 1);
+                        accumulate_quad_after_round1(xa0, ya0, a0, philox_round1_state(dp, ua, seed, rq), seed, layer);
+                        accumulate_quad_after_round1(xb0, yb0, b0, philox_round1_state(dp, ub, seed, rq), seed, layer);
+                        next_draw(dp);
+                        accumulate_quad_after_round1(xa1, ya1, a1, philox_round1_state(dp, ua, seed, rq), seed, layer);
+                        accumulate_quad_after_round1(xb1, yb1, b1, philox_round1_state(dp, ub, seed, rq), seed, layer);
+                        next_draw(dp);
+                    }
+                    if (j < n) {
+                        const float a0 = __shfl_sync(0xffffffffu, rva, j), b0 = __shfl_sync(0xffffffffu, rvb, j);
+                        accumulate_quad_after_round1(xa0, ya0, a0, philox_round1_state(dp, ua, seed, rq), seed, layer);
+                        accumulate_quad_after_round1(xb0, yb0, b0, philox_round1_state(dp, ub, seed, rq), seed, layer);
+                        next_draw(dp);
+                    }
                 }
-                if (k < nd) {
-                    accumulate_quad(xa0, ya0, __ldg(ra + static_cast<size_t>(k) * T), seed, layer, draw_begin + k, t0, quad);
-                    accumulate_quad(xb0, yb0, __ldg(rb + static_cast<size_t>(k) * T), seed, layer, draw_begin + k, t1, quad);
-                }
-            } else if (v0) {
-                for (; k + 2 <= nd; k += 2) {
-                    const float a0 = __ldg(ra + static_cast<size_t>(k) * T), a1 = __ldg(ra + static_cast<size_t>(k + 1) * T);
-                    accumulate_quad(xa0, ya0, a0, seed, layer, draw_begin + k, t0, quad);
-                    accumulate_quad(xa1, ya1, a1, seed, layer, draw_begin + k + 1, t0, quad);
-                }
-                if (k < nd)
-                    accumulate_quad(xa0, ya0, __ldg(ra + static_cast<size_t>(k) * T), seed, layer, draw_begin + k, t0, quad);
             }
             // g in the standalone reduction's order: (even draws + odd draws) * scale
             const float4 ga = make_float4((xa0.x + xa1.x) * scale, (ya0.x + ya1.x) * scale,
@@ -263,7 +299,14 @@ fused_estimate_kernel(const __grid_constant__ CUtensorMap map_x, const float* __
             *abort_flag = 1;
         }
         // ---------------- epilogue: TMEM -> fp32 partial row block of this token split
-        bool have = ok && n_stages > 0 && wait_or_abort(acc_full, 0, abort_flag, kProduceWaitLimit);
+        bool have = false;
+        if (ok && n_stages > 0) {
+            have = wait_or_abort_ns(acc_full, 0, abort_flag, produce_limit);
+            if (!have) {                               // this split's row block stays unwritten: say so
+                atomicExch(status, kStatusTimeout);
+                *abort_flag = 1;
+            }
+        }
         have = __all_sync(0xffffffffu, have);
         const int quarter = warp & 3;                 // the TMEM lane quarter this warp may read
         const int idx = pw >> 2;                      // 0 .. kProducerWarps/4 - 1 within the quarter
@@ -347,7 +390,7 @@ cudaError_t launch_fused_estimate(const float* r, int T, int d_out, const void* 
     const float scale = static_cast<float>(-1.0 / (static_cast<double>(nz.K_total) * nz.sigma));
     auto* partial = static_cast<float*>(scratch);
     fused_estimate_kernel<<<static_cast<unsigned>(tiles_m * sp.n_splits), kFusedThreads, L.bytes, stream>>>(
-        mx, r, T, d_out, d_in, nz.seed, nz.layer, nz.draw_begin, static_cast<int>(nz.draw_count), scale,
+        mx, r, T, d_out, d_in, nz.seed, nz.layer, nz.draw_begin, nz.token_begin, static_cast<int>(nz.draw_count), scale,
         sp.tokens_per_split, partial, g_hat, status);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -27,9 +27,11 @@ __device__ __forceinline__ float load_as_float<__nv_bfloat16>(const __nv_bfloat1
     return __bfloat162float(*p);
 }
 
-template <typename T, bool AK, bool BK>
+// A and B may differ in type (fp32 or bf16): every element is widened to fp32
+// exactly before the fp32 products.
+template <typename TA, typename TB, bool AK, bool BK>
 __global__ void __launch_bounds__(256)
-gemm_simt_kernel(const T* __restrict__ A, int lda, const T* __restrict__ B, int ldb, int M, int N,
+gemm_simt_kernel(const TA* __restrict__ A, int lda, const TB* __restrict__ B, int ldb, int M, int N,
                  int K, int k_per_split, float* __restrict__ C, int ldc, int accumulate,
                  float* __restrict__ partial) {
     __shared__ float As[kStep][kTile + 4];
@@ -108,15 +110,15 @@ __global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __r
         dst[i] = __float2bfloat16_rn(src[i]);
 }
 
-template <typename T>
-cudaError_t launch_typed(const T* A, bool ak, int lda, const T* B, bool bk, int ldb, int M, int N, int K,
+template <typename TA, typename TB>
+cudaError_t launch_typed(const TA* A, bool ak, int lda, const TB* B, bool bk, int ldb, int M, int N, int K,
                          float* C, int ldc, int accumulate, float* partial, int splits, cudaStream_t st) {
     const int kps = static_cast<int>(ceil_div(ceil_div(K, splits), kStep) * kStep);
     const dim3 grid(static_cast<unsigned>(ceil_div(N, kTile)), static_cast<unsigned>(ceil_div(M, kTile)),
                     static_cast<unsigned>(splits));
     float* part = splits > 1 ? partial : nullptr;
 #define DUST_SIMT_LAUNCH(AKV, BKV) \
-    gemm_simt_kernel<T, AKV, BKV><<<grid, 256, 0, st>>>(A, lda, B, ldb, M, N, K, kps, C, ldc, accumulate, part)
+    gemm_simt_kernel<TA, TB, AKV, BKV><<<grid, 256, 0, st>>>(A, lda, B, ldb, M, N, K, kps, C, ldc, accumulate, part)
     if (ak && bk) DUST_SIMT_LAUNCH(true, true);
     else if (ak && !bk) DUST_SIMT_LAUNCH(true, false);
     else if (!ak && bk) DUST_SIMT_LAUNCH(false, true);
@@ -142,12 +144,28 @@ int gemm_simt_splits(int M, int N, int K) {
 cudaError_t launch_gemm_simt(const void* A, bool a_kmajor, int lda, const void* B, bool b_kmajor, int ldb,
                              dust_dtype dt, int M, int N, int K, float* C, int ldc, int accumulate,
                              float* partial, int splits, cudaStream_t stream) {
-    if (dt == DUST_F32)
-        return launch_typed(static_cast<const float*>(A), a_kmajor, lda, static_cast<const float*>(B), b_kmajor,
-                            ldb, M, N, K, C, ldc, accumulate, partial, splits, stream);
-    return launch_typed(static_cast<const __nv_bfloat16*>(A), a_kmajor, lda,
-                        static_cast<const __nv_bfloat16*>(B), b_kmajor, ldb, M, N, K, C, ldc, accumulate,
-                        partial, splits, stream);
+    return launch_gemm_simt_mixed(A, dt, a_kmajor, lda, B, dt, b_kmajor, ldb, M, N, K, C, ldc, accumulate, partial,
+                                  splits, stream);
+}
+
+cudaError_t launch_gemm_simt_mixed(const void* A, dust_dtype a_dt, bool a_kmajor, int lda, const void* B,
+                                   dust_dtype b_dt, bool b_kmajor, int ldb, int M, int N, int K, float* C, int ldc,
+                                   int accumulate, float* partial, int splits, cudaStream_t stream) {
+    using bf = __nv_bfloat16;
+    const auto* af = static_cast<const float*>(A);
+    const auto* ab = static_cast<const bf*>(A);
+    const auto* bf32 = static_cast<const float*>(B);
+    const auto* bb = static_cast<const bf*>(B);
+    if (a_dt == DUST_F32 && b_dt == DUST_F32)
+        return launch_typed(af, a_kmajor, lda, bf32, b_kmajor, ldb, M, N, K, C, ldc, accumulate, partial, splits,
+                            stream);
+    if (a_dt == DUST_F32)
+        return launch_typed(af, a_kmajor, lda, bb, b_kmajor, ldb, M, N, K, C, ldc, accumulate, partial, splits,
+                            stream);
+    if (b_dt == DUST_F32)
+        return launch_typed(ab, a_kmajor, lda, bf32, b_kmajor, ldb, M, N, K, C, ldc, accumulate, partial, splits,
+                            stream);
+    return launch_typed(ab, a_kmajor, lda, bb, b_kmajor, ldb, M, N, K, C, ldc, accumulate, partial, splits, stream);
 }
 
 cudaError_t launch_splitk_reduce(const float* partial, int splits, int M, int N, float* C, int ldc,

@@ -9,17 +9,24 @@
 //   a2: C[T][V] = sum_k X[t][k] W[v][k]: both operands are K-major.
 //
 // Tile 128 x BN (BN in {64, 128, 256}), 64-deep k blocks in a 4-stage ring.
-// One CTA of 4 warps per output tile and k slice:
+// The kernel is persistent: one CTA of 10 warps per SM walks the work units
+// (output tile, k slice) in a grid-stride loop, and the roles are split by warp:
 //   warp 0, one lane: TMA producer (cp.async.bulk.tensor, 128-byte swizzle,
-//           each CTA loads its own tiles), one mbarrier per stage with expected bytes;
+//           each CTA loads its own tiles into its own shared memory), one
+//           mbarrier per stage with the expected bytes;
 //   warp 1, one lane: MMA issuer, 4 x tcgen05.mma (M = 128, N = BN, K = 16)
 //           per stage, tcgen05.commit frees the stage; warp 1 also allocates
-//           and frees the TMEM accumulator (BN fp32 columns);
-//   warps 0-3: epilogue, tcgen05.ld of its 32 TMEM lanes (rows), fp32 stores.
+//           and frees TMEM: two BN-column fp32 accumulators (2 BN columns), so
+//           that unit i's epilogue overlaps unit i+1's main loop;
+//   warps 2-9: epilogue, two warps per TMEM lane quarter taking alternate
+//           32-column blocks: tcgen05.ld of the warp's 32 TMEM lanes (rows),
+//           an xor-swizzled 32 x 32 shared-memory transpose, then row-segment
+//           fp32 stores; the warps release the accumulator buffer afterwards.
 // Split over k writes fp32 partial tiles that a second kernel sums in a fixed
 // order (deterministic).  Every mbarrier wait is bounded: when a bound runs
-// out the kernel records the workspace status word, drains its own copies and
-// MMAs (bounded too), frees TMEM and returns.
+// out the role records the workspace status word, raises the CTA's abort flag
+// (which ends the other roles' waits), drains its own copies and MMAs
+// (bounded too), frees TMEM and returns.
 #include <cuda.h>
 
 #include <mutex>
@@ -225,7 +232,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             const Unit w = unit_of(u, tiles_m, tiles_n, BN, K, k_per_split);
             const int buf = tcount & 1;
             bool have = mbar_wait_or_abort(&tfull[buf], (tcount >> 1) & 1, abort_flag);
-            if (!__all_sync(0xffffffffu, have)) break;
+            if (!__all_sync(0xffffffffu, have)) {
+                // this unit's tile stays unwritten: record it (another role may
+                // have done so already; the word and the flag only ever get set)
+                if (lane == 0) {
+                    atomicExch(status, kStatusTimeout);
+                    *abort_flag = 1;
+                }
+                break;
+            }
             tc_fence_after();
             have = w.nk > 0;
             const int split = u / (tiles_m * tiles_n);

@@ -105,9 +105,10 @@ constexpr int kHeadWarps = 4;   // tokens per block
 template <int QPL, int TIER, int WPT>
 __global__ void __launch_bounds__(32 * kHeadWarps)
 head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
-                  const int32_t* __restrict__ targets, int T, int V, int Vc, uint32_t seed, uint32_t layer,
-                  uint32_t draw_begin, int nd, float sigma, float scale, float* __restrict__ c_out,
-                  float* __restrict__ g, __nv_bfloat16* __restrict__ g16, int accumulate) {
+                  const int32_t* __restrict__ targets, int T, int V, int Vc, int chunk0, int ldg, uint32_t seed,
+                  uint32_t layer, uint32_t draw_begin, uint32_t tok0, int nd, float sigma, float scale,
+                  float* __restrict__ c_out, float* __restrict__ g, __nv_bfloat16* __restrict__ g16,
+                  int accumulate) {
     constexpr int kTPB = kHeadWarps / WPT;        // tokens per block
     constexpr int kSub = 128 * QPL;               // vocab ids per warp
     // the softmax probabilities of each warp's ids (times sigma for the series
@@ -120,7 +121,8 @@ head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
     const int ts = warp / WPT, part = warp % WPT;
     const int t = blockIdx.x * kTPB + ts;
     if (t >= T) return;                           // the token's warps leave together
-    const int chunk = blockIdx.y;
+    const int cidx = blockIdx.y;                  // chunk of this call's range: g's column block, c's row block
+    const int chunk = chunk0 + cidx;              // its vocabulary chunk
     const int v0 = chunk * Vc + part * kSub;      // first id of this warp
     const float* zt = Z + static_cast<size_t>(t) * V;
     const float l = __ldg(lse + t);
@@ -155,7 +157,7 @@ head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
         float ay = 0.0f;
 #pragma unroll
         for (int k = 0; k < QPL; ++k) {
-            const Gauss4Pairs n = gauss4_pairs(seed, layer, draw, static_cast<uint32_t>(t), quad0 + 32u * k, 0);
+            const Gauss4Pairs n = gauss4_pairs(seed, layer, draw, tok0 + static_cast<uint32_t>(t), quad0 + 32u * k, 0);
             ae[k] = n.even;
             ao[k] = n.odd;
             const float4 pk = p[lane + 32 * k];
@@ -183,7 +185,7 @@ head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
             }
         }
         const float c = log1pf(S) - (in_chunk ? sy : 0.0f);
-        if (c_out != nullptr && lane == 0 && part == 0) c_out[(static_cast<size_t>(chunk) * nd + i) * T + t] = c;
+        if (c_out != nullptr && lane == 0 && part == 0) c_out[(static_cast<size_t>(cidx) * nd + i) * T + t] = c;
         const float2 cc = splat(c);
 #pragma unroll
         for (int k = 0; k < QPL; ++k) {
@@ -194,7 +196,7 @@ head_chunk_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
 
 #pragma unroll
     for (int k = 0; k < QPL; ++k) {
-        const size_t off = static_cast<size_t>(t) * V + v0 + 4 * (lane + 32 * k);
+        const size_t off = static_cast<size_t>(t) * ldg + cidx * Vc + part * kSub + 4 * (lane + 32 * k);
         float4 out = make_float4(ge[k].x * scale, go[k].x * scale, ge[k].y * scale, go[k].y * scale);
         float4* gp = reinterpret_cast<float4*>(g + off);
         if (accumulate) {
@@ -232,13 +234,14 @@ namespace {
 
 template <int QPL, int WPT>
 void launch_qw(int tier, dim3 grid, cudaStream_t st, const float* Z, const float* lse, const int32_t* targets, int T,
-               int V, int Vc, const dust_noise& nz, float scale, float* c_out, float* g, __nv_bfloat16* g16,
-               int accumulate) {
+               int V, int Vc, int chunk0, const dust_noise& nz, float scale, float* c_out, float* g,
+               __nv_bfloat16* g16, int accumulate) {
     const int nd = static_cast<int>(nz.draw_count);
-#define DUST_HEAD_TIER(TIER_)                                                                               \
-    head_chunk_kernel<QPL, TIER_, WPT><<<grid, 32 * kHeadWarps, 0, st>>>(Z, lse, targets, T, V, Vc, nz.seed,  \
-                                                                         nz.layer, nz.draw_begin, nd, nz.sigma, \
-                                                                         scale, c_out, g, g16, accumulate)
+    const int ldg = static_cast<int>(grid.y) * Vc;
+#define DUST_HEAD_TIER(TIER_)                                                                                \
+    head_chunk_kernel<QPL, TIER_, WPT><<<grid, 32 * kHeadWarps, 0, st>>>(                                    \
+        Z, lse, targets, T, V, Vc, chunk0, ldg, nz.seed, nz.layer, nz.draw_begin, nz.token_begin, nd, nz.sigma, \
+        scale, c_out, g, g16, accumulate)
     if (tier == 2) DUST_HEAD_TIER(2);
     else if (tier == 1) DUST_HEAD_TIER(1);
     else DUST_HEAD_TIER(0);
@@ -248,18 +251,18 @@ void launch_qw(int tier, dim3 grid, cudaStream_t st, const float* Z, const float
 }  // namespace
 
 cudaError_t launch_head_chunks(const float* Z, const float* lse, const int32_t* targets, int T, int V, int Vc,
-                               const dust_noise& nz, float* c_out, float* g, void* g_bf16, int accumulate,
-                               cudaStream_t stream) {
+                               int chunk_begin, int chunk_count, const dust_noise& nz, float* c_out, float* g,
+                               void* g_bf16, int accumulate, cudaStream_t stream) {
     if (!head_chunk_supported(Vc)) return cudaErrorNotSupported;
     const int wpt = Vc <= 1024 ? 1 : (Vc <= 2048 ? 2 : 4);
     const int qpl = Vc / (128 * wpt);
-    const dim3 grid(static_cast<unsigned>(ceil_div(T, kHeadWarps / wpt)), static_cast<unsigned>(V / Vc));
+    const dim3 grid(static_cast<unsigned>(ceil_div(T, kHeadWarps / wpt)), static_cast<unsigned>(chunk_count));
     // |a| < 5.66 for every draw the generator produces (see expm1_series)
     const int tier = nz.sigma <= 0.01f ? 2 : (nz.sigma <= 0.02f ? 1 : 0);
     const float scale = static_cast<float>(-1.0 / (static_cast<double>(nz.K_total) * nz.sigma));
     auto* g16 = static_cast<__nv_bfloat16*>(g_bf16);
-#define DUST_HEAD_QW(Q, W)                                                                            \
-    launch_qw<Q, W>(tier, grid, stream, Z, lse, targets, T, V, Vc, nz, scale, c_out, g, g16, accumulate)
+#define DUST_HEAD_QW(Q, W)                                                                                   \
+    launch_qw<Q, W>(tier, grid, stream, Z, lse, targets, T, V, Vc, chunk_begin, nz, scale, c_out, g, g16, accumulate)
     if (wpt == 1) {
         switch (qpl) {
             case 1: DUST_HEAD_QW(1, 1); break;

@@ -44,6 +44,10 @@ cudaError_t launch_synth_costs(const float* u, int T, int d_out, const dust_nois
 cudaError_t launch_gemm_simt(const void* A, bool a_kmajor, int lda, const void* B, bool b_kmajor,
                              int ldb, dust_dtype dt, int M, int N, int K, float* C, int ldc,
                              int accumulate, float* partial, int splits, cudaStream_t stream);
+// the same with A and B of different types (each widened to fp32 exactly)
+cudaError_t launch_gemm_simt_mixed(const void* A, dust_dtype a_dt, bool a_kmajor, int lda, const void* B,
+                                   dust_dtype b_dt, bool b_kmajor, int ldb, int M, int N, int K, float* C, int ldc,
+                                   int accumulate, float* partial, int splits, cudaStream_t stream);
 int gemm_simt_splits(int M, int N, int K);
 // C (+)= sum_s partial[s]  (fixed order), C [M][N] leading dim ldc
 cudaError_t launch_splitk_reduce(const float* partial, int splits, int M, int N, float* C, int ldc,
@@ -68,6 +72,9 @@ int device_sm_count();
 // d_in a multiple of 64 up to 512.  scratch holds fused_estimate_scratch()
 // bytes (fp32 partial G row blocks, one per token split).
 bool fused_estimate_supported(int d_in, int d_out);
+// draws per call of the fused kernel: its waits on a stage's production are
+// bounded by a time budget that grows with the draw count
+constexpr uint32_t kFusedMaxDraws = 1u << 20;
 size_t fused_estimate_scratch(int T, int d_in, int d_out);
 cudaError_t launch_fused_estimate(const float* r, int T, int d_out, const void* X, int d_in, const dust_noise& nz,
                                   float* G, int accumulate, float* g_hat, void* scratch, uint32_t* status,
@@ -77,9 +84,11 @@ cudaError_t launch_fused_estimate(const float* r, int T, int d_out, const void* 
 cudaError_t launch_row_stats(const float* Z, const int32_t* targets, int T, int V, float* lse,
                              float* ell, cudaStream_t stream);
 bool head_chunk_supported(int Vc);
+// chunks [chunk_begin, chunk_begin + chunk_count) of width Vc; g and g_bf16 are
+// [T][chunk_count Vc] (the range's columns), c_out [chunk_count][draw_count][T]
 cudaError_t launch_head_chunks(const float* Z, const float* lse, const int32_t* targets, int T,
-                               int V, int Vc, const dust_noise& nz, float* c_out, float* g,
-                               void* g_bf16, int accumulate, cudaStream_t stream);
+                               int V, int Vc, int chunk_begin, int chunk_count, const dust_noise& nz,
+                               float* c_out, float* g, void* g_bf16, int accumulate, cudaStream_t stream);
 
 // harness: toy causal suffix (toy_suffix.cu)
 size_t toy_suffix_workspace_bytes(int draw_count, int T, int d, int dh, int V);
@@ -106,10 +115,12 @@ cudaError_t launch_causal_attention(const float* q, const float* k, const float*
 
 // attention-internal scoring (attention_scoring.cu)
 size_t attention_scoring_workspace_bytes(int draw_count, int T, int d, int dh);
+// which: 0 q, 1 k, 2 v, 3 the gate's pre-activation Y Wg^T, 4 the value
+// embedding E; the values are Y Wv^T + s(Y Wg^T) E (Wg, E nullable)
 cudaError_t run_attention_internal_costs(const float* Y, int T, int d, const int32_t* offs, int n_seq,
-                                         const float* Wq, const float* Wk, const float* Wv, const float* Wo, int dh,
-                                         int which, const float* G, const dust_noise& nz, float* c, void* ws,
-                                         cudaStream_t st);
+                                         const float* Wq, const float* Wk, const float* Wv, const float* Wo,
+                                         const float* Wg, const float* E, int dh, int which, const float* G,
+                                         const dust_noise& nz, float* c, void* ws, cudaStream_t st);
 
 // fp32 -> bf16 (RNE) copy
 cudaError_t launch_to_bf16(const float* src, void* dst, size_t n, cudaStream_t stream);

@@ -7,14 +7,19 @@
 // Design (B200): the work is K x T x d_out Gaussians, each regenerated from its
 // coordinates (noise.cuh) and consumed by one FMA; nothing K x T x d is ever
 // stored, and the only HBM traffic is r (4 bytes per draw x token, a warp-wide
-// broadcast) and g (written once).  The kernel is therefore bound by the SM
-// issue rate, not by HBM.  One thread owns (token t, channel quad q): a single
-// Philox call per draw yields its 4 channels, whose two Box-Muller pairs run
-// in lock-step on the packed fp32 pipes, so the counter words that do not
-// depend on the draw (first-round product of the quad, key schedule) are
-// hoisted out of the draw loop.  Two draws per iteration give the scheduler two
-// independent Philox chains.  Blocks are 256 threads: quads along x (coalesced
-// 128-bit stores of g), tokens along y.
+// broadcast) and g (written once).  The kernel is therefore bound by the SM's
+// fp32/integer-multiply datapath, not by HBM.  One thread owns (token t,
+// channel quad q): a single Philox call per draw yields its 4 channels, whose
+// two Box-Muller pairs run in lock-step on the packed fp32 pipes.  Work that
+// does not change along the draw loop leaves it: the key schedule, and the
+// quad's half of Philox round 1 (philox_round1_quad); the draw's half is the
+// 64-bit product M1 d, stepped by an add from one draw to the next instead of a
+// wide multiply on the busiest datapath.  A warp shares its token, so lane j
+// loads r for draw k0 + j once per 32 draws and the loop takes them by shuffle,
+// with no per-draw address arithmetic.  Four draws per iteration alternate
+// between two accumulator pairs (even and odd draws), which gives the scheduler
+// independent chains and fixes the summation order.  Blocks are 256 threads:
+// quads along x (coalesced 128-bit stores of g), tokens along y.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -32,24 +37,50 @@ namespace {
 template <bool kVec, bool kAcc, bool kG16>
 __global__ void __launch_bounds__(256)
 layer_estimate_kernel(const float* __restrict__ r, int T, int d_out, int nq, uint32_t seed,
-                      uint32_t layer, uint32_t draw_begin, int nd, float scale,
+                      uint32_t layer, uint32_t draw_begin, uint32_t tok0, int nd, float scale,
                       float* __restrict__ g, __nv_bfloat16* __restrict__ g16) {
-    const int q = blockIdx.x * blockDim.x + threadIdx.x;
-    if (q >= nq) return;
+    // a warp shares one token (blockDim.x >= 32): lane j loads the r of draw
+    // k0 + j and the draws of a 32-draw group are passed round by shuffles
+    const int q_raw = blockIdx.x * blockDim.x + threadIdx.x;
+    const int lane = threadIdx.x & 31;
+    if (__all_sync(0xffffffffu, q_raw >= nq)) return;
+    const int q = q_raw < nq ? q_raw : nq - 1;
+    const uint2 rq = philox_round1_quad(static_cast<uint32_t>(q), 0u, layer);
     for (int t = blockIdx.y * blockDim.y + threadIdx.y; t < T; t += gridDim.y * blockDim.y) {
         float2 xz0 = splat(0.0f), yw0 = splat(0.0f), xz1 = splat(0.0f), yw1 = splat(0.0f);
         const float* rt = r + t;
-        int k = 0;
-        for (; k + 2 <= nd; k += 2) {
-            const float r0 = __ldg(rt + static_cast<size_t>(k) * T);
-            const float r1 = __ldg(rt + static_cast<size_t>(k + 1) * T);
-            accumulate_quad(xz0, yw0, r0, seed, layer, draw_begin + k, t, q);
-            accumulate_quad(xz1, yw1, r1, seed, layer, draw_begin + k + 1, t, q);
+        const uint32_t tok = tok0 + static_cast<uint32_t>(t);     // the token's global index: its noise
+        DrawProduct dp = draw_product(draw_begin);
+        for (int k0 = 0; k0 < nd; k0 += 32) {
+            const int n = nd - k0 < 32 ? nd - k0 : 32;
+            const float rv = lane < n ? __ldg(rt + static_cast<size_t>(k0 + lane) * T) : 0.0f;
+            int j = 0;
+            for (; j + 4 <= n; j += 4) {
+                const float r0 = __shfl_sync(0xffffffffu, rv, j), r1 = __shfl_sync(0xffffffffu, rv, j + 1);
+                const float r2 = __shfl_sync(0xffffffffu, rv, j + 2), r3 = __shfl_sync(0xffffffffu, rv, j + 3);
+                accumulate_quad_after_round1(xz0, yw0, r0, philox_round1_state(dp, tok, seed, rq), seed, layer);
+                next_draw(dp);
+                accumulate_quad_after_round1(xz1, yw1, r1, philox_round1_state(dp, tok, seed, rq), seed, layer);
+                next_draw(dp);
+                accumulate_quad_after_round1(xz0, yw0, r2, philox_round1_state(dp, tok, seed, rq), seed, layer);
+                next_draw(dp);
+                accumulate_quad_after_round1(xz1, yw1, r3, philox_round1_state(dp, tok, seed, rq), seed, layer);
+                next_draw(dp);
+            }
+            for (; j + 2 <= n; j += 2) {
+                const float r0 = __shfl_sync(0xffffffffu, rv, j), r1 = __shfl_sync(0xffffffffu, rv, j + 1);
+                accumulate_quad_after_round1(xz0, yw0, r0, philox_round1_state(dp, tok, seed, rq), seed, layer);
+                next_draw(dp);
+                accumulate_quad_after_round1(xz1, yw1, r1, philox_round1_state(dp, tok, seed, rq), seed, layer);
+                next_draw(dp);
+            }
+            if (j < n) {
+                const float r0 = __shfl_sync(0xffffffffu, rv, j);
+                accumulate_quad_after_round1(xz0, yw0, r0, philox_round1_state(dp, tok, seed, rq), seed, layer);
+                next_draw(dp);
+            }
         }
-        if (k < nd) {
-            const float r0 = __ldg(rt + static_cast<size_t>(k) * T);
-            accumulate_quad(xz0, yw0, r0, seed, layer, draw_begin + k, t, q);
-        }
+        if (q_raw >= nq) continue;
         float4 out = make_float4((xz0.x + xz1.x) * scale, (yw0.x + yw1.x) * scale,
                                  (xz0.y + xz1.y) * scale, (yw0.y + yw1.y) * scale);
         const size_t base = static_cast<size_t>(t) * d_out + 4 * static_cast<size_t>(q);
@@ -88,10 +119,12 @@ void launch_g16(bool with_g16, dim3 grid, dim3 block, cudaStream_t stream, const
     const int nd = static_cast<int>(nz.draw_count);
     if (with_g16)
         layer_estimate_kernel<kVec, kAcc, true><<<grid, block, 0, stream>>>(r, T, d_out, nq, nz.seed, nz.layer,
-                                                                            nz.draw_begin, nd, scale, g, g16);
+                                                                            nz.draw_begin, nz.token_begin, nd,
+                                                                            scale, g, g16);
     else
         layer_estimate_kernel<kVec, kAcc, false><<<grid, block, 0, stream>>>(r, T, d_out, nq, nz.seed, nz.layer,
-                                                                             nz.draw_begin, nd, scale, g, g16);
+                                                                             nz.draw_begin, nz.token_begin, nd,
+                                                                             scale, g, g16);
 }
 
 }  // namespace

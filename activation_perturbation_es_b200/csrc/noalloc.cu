@@ -12,7 +12,11 @@
 //
 // Costs and limits of the static array:
 //   - every GPU on which the library is loaded holds kNoAllocScratchBytes
-//     (16 MiB) for it until the process exits;
+//     (16 MiB for the rewards, plus 64 KiB for the chunk maps of the chunked
+//     scan) for it until the process exits;
+//   - the reward scan takes the same path as dust_layer_estimate's (per
+//     sequence, or over 1024-token chunks for few long sequences), so both
+//     entry points return the same bits;
 //   - draw_count * T must not exceed kNoAllocScratchFloats (4 Mi) when the
 //     scan is needed (gamma > 0); split the draws over several calls with
 //     accumulate = 1 otherwise (the estimate is linear in the draws);
@@ -27,6 +31,9 @@
 // stand-in symbol, not a device address.  The device address is looked up with
 // cudaGetSymbolAddress once per device, with that device current, on the first
 // call made on that device; make that first call before any stream capture.
+// The address is cached for the life of the process: after cudaDeviceReset of
+// a device it is stale, and this entry point must not be used on that device
+// again.
 #include <cmath>
 #include <cstdio>
 #include <mutex>
@@ -38,11 +45,15 @@ namespace dust {
 
 namespace {
 
-constexpr size_t kNoAllocScratchFloats = size_t(1) << 22;
-constexpr size_t kNoAllocScratchBytes = kNoAllocScratchFloats * sizeof(float);
-static_assert(kNoAllocScratchBytes == (size_t(16) << 20), "16 MiB of static scratch");
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 22;           // the rewards r: 16 MiB
+// The chunked scan runs only when draws x sequences < 4 x 148 (so draw_count
+// < 592), and then needs 12 bytes per (draw, 1024-token chunk): at most
+// (4 Mi / 1024 + 592) x 12 bytes < 64 KiB within the rewards' limit.
+constexpr size_t kNoAllocChunkFloats = size_t(1) << 14;             // 64 KiB
+constexpr size_t kNoAllocScratchBytes = (kNoAllocScratchFloats + kNoAllocChunkFloats) * sizeof(float);
+static_assert(kNoAllocScratchFloats * sizeof(float) == (size_t(16) << 20), "16 MiB of static scratch for r");
 
-static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats + kNoAllocChunkFloats];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
@@ -85,6 +96,7 @@ extern "C" dust_status dust_layer_estimate_noalloc(const float* c, int T, int d_
         return reject(DUST_ERR_INVALID_ARG, "noise: draw_count and K_total must be > 0, sigma finite and > 0");
     if (static_cast<unsigned long long>(nz.draw_begin) + nz.draw_count > (1ull << 32))
         return reject(DUST_ERR_INVALID_ARG, "draw_begin + draw_count exceeds 2^32");
+    if (nz.token_begin > 0x7FFFFFFFu) return reject(DUST_ERR_INVALID_ARG, "token_begin must be < 2^31");
     if (T <= 0 || d_out <= 0) return reject(DUST_ERR_INVALID_ARG, "T and d_out must be > 0 (T=%lld, d_out=%lld)", T, d_out);
     if (!(gamma >= 0.0f && gamma <= 1.0f)) return reject(DUST_ERR_INVALID_ARG, "gamma must be in [0, 1]");
     if (c == nullptr || g_hat == nullptr) return reject(DUST_ERR_INVALID_ARG, "c and g_hat must not be NULL");
@@ -105,8 +117,15 @@ extern "C" dust_status dust_layer_estimate_noalloc(const float* c, int T, int d_
             return reject(DUST_ERR_INVALID_ARG, "draws x sequences must be < 2^31");
         float* scratch = nullptr;
         cudaError_t e = scratch_address(&scratch);
+        const int K = static_cast<int>(nz.draw_count);
+        // the scan dust_layer_estimate would run (same bits); the chunk maps live
+        // behind the rewards (their size always fits, see kNoAllocChunkFloats)
+        const bool chunks = reward_scan_prefers_chunks(K, T, n_seq) &&
+                            reward_scan_chunks_workspace(K, T) <= kNoAllocChunkFloats * sizeof(float);
         if (e == cudaSuccess)
-            e = launch_reward_scan(c, scratch, static_cast<int>(nz.draw_count), T, seq_offsets, n_seq, gamma, st);
+            e = chunks ? launch_reward_scan_chunks(c, scratch, K, T, seq_offsets, n_seq, gamma,
+                                                   scratch + kNoAllocScratchFloats, st)
+                       : launch_reward_scan(c, scratch, K, T, seq_offsets, n_seq, gamma, st);
         if (e != cudaSuccess) return record_error(DUST_ERR_CUDA, cudaGetErrorString(e));
         r = scratch;
     }

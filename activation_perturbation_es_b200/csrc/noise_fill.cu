@@ -14,7 +14,7 @@ namespace dust {
 namespace {
 
 __global__ void noise_fill_kernel(uint32_t seed, uint32_t layer, uint32_t stream_id,
-                                  uint32_t draw_begin, int nd, int t0, int n_tok, int j0, int n_ch,
+                                  uint32_t draw_begin, int nd, uint32_t tok0, int t0, int n_tok, int j0, int n_ch,
                                   float* __restrict__ out) {
     const long long total = static_cast<long long>(nd) * n_tok * n_ch;
     for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
@@ -24,7 +24,7 @@ __global__ void noise_fill_kernel(uint32_t seed, uint32_t layer, uint32_t stream
         const int t = static_cast<int>(rest % n_tok);
         const int k = static_cast<int>(rest / n_tok);
         const uint32_t ch = static_cast<uint32_t>(j0 + j);
-        const float4 a = gauss4(seed, layer, draw_begin + k, static_cast<uint32_t>(t0 + t), ch >> 2, stream_id);
+        const float4 a = gauss4(seed, layer, draw_begin + k, tok0 + static_cast<uint32_t>(t0 + t), ch >> 2, stream_id);
         const uint32_t w = ch & 3u;
         out[idx] = w == 0 ? a.x : (w == 1 ? a.y : (w == 2 ? a.z : a.w));
     }
@@ -55,7 +55,8 @@ __global__ void box_muller_words_kernel(const uint32_t* __restrict__ a, const ui
 // results are transposed through shared memory into 32-byte runs of c.
 __global__ void __launch_bounds__(256)
 synth_costs_kernel(const float* __restrict__ u, int T, int d_out, uint32_t seed, uint32_t layer,
-                   uint32_t draw_begin, int nd, float sigma, float eps_scale, float* __restrict__ c) {
+                   uint32_t draw_begin, uint32_t tok0, int nd, float sigma, float eps_scale,
+                   float* __restrict__ c) {
     __shared__ float tile[32][9];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int s = blockIdx.x * 8 + warp;
@@ -77,13 +78,13 @@ synth_costs_kernel(const float* __restrict__ u, int T, int d_out, uint32_t seed,
                 uv.z = j + 2 < d_out ? __ldg(us + j + 2) : 0.0f;
                 uv.w = j + 3 < d_out ? __ldg(us + j + 3) : 0.0f;
             }
-            const float4 a = gauss4(seed, layer, draw, static_cast<uint32_t>(s), static_cast<uint32_t>(q), 0);
+            const float4 a = gauss4(seed, layer, draw, tok0 + static_cast<uint32_t>(s), static_cast<uint32_t>(q), 0);
             dot0 = __fmaf_rn(uv.x, a.x, dot0);
             dot1 = __fmaf_rn(uv.y, a.y, dot1);
             dot0 = __fmaf_rn(uv.z, a.z, dot0);
             dot1 = __fmaf_rn(uv.w, a.w, dot1);
         }
-        const float eps = gauss4(seed, layer, draw, static_cast<uint32_t>(s), 0, 1).x;
+        const float eps = gauss4(seed, layer, draw, tok0 + static_cast<uint32_t>(s), 0, 1).x;
         val = sigma * (dot0 + dot1) + eps_scale * eps;
     }
     tile[lane][warp] = val;
@@ -101,7 +102,7 @@ cudaError_t launch_noise_fill(const dust_noise& nz, uint32_t stream_id, int t0, 
     if (total == 0) return cudaSuccess;
     const long long blocks = ceil_div(total, 256);
     noise_fill_kernel<<<static_cast<unsigned>(blocks < 65536 ? blocks : 65536), 256, 0, stream>>>(
-        nz.seed, nz.layer, stream_id, nz.draw_begin, static_cast<int>(nz.draw_count), t0, n_tok, j0,
+        nz.seed, nz.layer, stream_id, nz.draw_begin, static_cast<int>(nz.draw_count), nz.token_begin, t0, n_tok, j0,
         n_ch, out);
     return cudaGetLastError();
 }
@@ -118,7 +119,7 @@ cudaError_t launch_box_muller_words(const uint32_t* a, const uint32_t* b, long l
 cudaError_t launch_synth_costs(const float* u, int T, int d_out, const dust_noise& nz, float eps_scale,
                                float* c, cudaStream_t stream) {
     const dim3 grid(static_cast<unsigned>(ceil_div(T, 8)), static_cast<unsigned>(ceil_div(nz.draw_count, 32)));
-    synth_costs_kernel<<<grid, 256, 0, stream>>>(u, T, d_out, nz.seed, nz.layer, nz.draw_begin,
+    synth_costs_kernel<<<grid, 256, 0, stream>>>(u, T, d_out, nz.seed, nz.layer, nz.draw_begin, nz.token_begin,
                                                  static_cast<int>(nz.draw_count), nz.sigma, eps_scale, c);
     return cudaGetLastError();
 }

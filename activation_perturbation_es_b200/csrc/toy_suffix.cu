@@ -20,9 +20,10 @@ namespace dust {
 
 namespace {
 
-// rows [b][t][j]: Y + sigma a(draw_of[b], t, j), or Y for the clean row
+// rows [b][t][j]: Y + sigma a(draw_of[b], tok0 + t, j), or Y for the clean row
 __global__ void perturb_kernel(const float* __restrict__ Y, int T, int d, uint32_t seed, uint32_t layer,
-                               uint32_t first_draw, int clean_first, int nb, float sigma, float* __restrict__ out) {
+                               uint32_t tok0, uint32_t first_draw, int clean_first, int nb, float sigma,
+                               float* __restrict__ out) {
     const int nq = d / 4;
     const long long total = static_cast<long long>(nb) * T * nq;
     for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
@@ -34,7 +35,7 @@ __global__ void perturb_kernel(const float* __restrict__ Y, int T, int d, uint32
         float4 y = __ldg(reinterpret_cast<const float4*>(Y + static_cast<size_t>(t) * d) + q);
         if (!(clean_first && b == 0)) {
             const uint32_t draw = first_draw + static_cast<uint32_t>(b - clean_first);
-            const float4 a = gauss4(seed, layer, draw, static_cast<uint32_t>(t), static_cast<uint32_t>(q), 0);
+            const float4 a = gauss4(seed, layer, draw, tok0 + static_cast<uint32_t>(t), static_cast<uint32_t>(q), 0);
             y.x += sigma * a.x; y.y += sigma * a.y; y.z += sigma * a.z; y.w += sigma * a.w;
         }
         reinterpret_cast<float4*>(out + static_cast<size_t>(b * static_cast<long long>(T) + t) * d)[q] = y;
@@ -200,8 +201,8 @@ cudaError_t run_toy_suffix(const float* Y, int T, int d, const int32_t* offs, in
         const uint32_t first_draw = nz.draw_begin + static_cast<uint32_t>(r0 == 0 ? 0 : r0 - 1);
         const long long rows = static_cast<long long>(nb) * T;
         const int M = static_cast<int>(rows);
-        perturb_kernel<<<blocks_for(rows * (d / 4), 256), 256, 0, st>>>(Y, T, d, nz.seed, nz.layer, first_draw,
-                                                                          clean_first, nb, nz.sigma, yt);
+        perturb_kernel<<<blocks_for(rows * (d / 4), 256), 256, 0, st>>>(Y, T, d, nz.seed, nz.layer, nz.token_begin,
+                                                                          first_draw, clean_first, nb, nz.sigma, yt);
         if ((e = cudaGetLastError()) != cudaSuccess) break;
         const float* Ws[3] = {Wq, Wk, Wv};
         float* outs[3] = {q, k, v};

@@ -1,15 +1,22 @@
 """Data-parallel plumbing for the estimator (host side, torch.distributed).
 
-The estimator shards two ways without changing what it computes:
+The estimator shards three ways without changing what it computes:
   * by sequences (data parallel): each rank owns whole sequences -- the reward
-    scan never crosses a sequence -- and the weight estimates of all ranks are
-    summed, G_W = sum_t g_t x_t^T over the global batch (cnblogs Dust
+    scan never crosses a sequence -- and passes the global index of its first
+    token as the noise's token_begin, so every token draws the noise it would
+    draw in one run over the whole batch; the weight estimates of all ranks
+    are summed, G_W = sum_t g_t x_t^T over the global batch (cnblogs Dust
     explainer, credit-assignment section, weight equation);
   * by draws: each rank takes a contiguous range of the global draw indices
     and scales by the whole population K_total, so the sum over ranks of the
     partial estimates is the K-draw estimate (error equation, linear in the
-    draws).
-Either way the only exchange is one sum all-reduce per step.
+    draws);
+  * the LM head by vocabulary chunk (the interference-suppression section's
+    third measure perturbs one chunk per pass): each rank runs a contiguous
+    range of the chunk passes; their g columns and G_W rows are disjoint, so
+    the rows are gathered, not summed.
+The exchange is one sum all-reduce per step (and one gather of the head's
+rows when the head is split by chunk).
 """
 from __future__ import annotations
 
@@ -30,6 +37,34 @@ def sequence_range(n_seq: int, world: int, rank: int) -> tuple[int, int]:
     if not 0 <= rank < world:
         raise ValueError("rank out of range")
     return n_seq * rank // world, n_seq * (rank + 1) // world
+
+
+def chunk_range(n_chunks: int, world: int, rank: int) -> tuple[int, int]:
+    """(chunk_begin, chunk_count) of `rank` when n_chunks vocabulary chunks are
+    split over `world` ranks (chunk_count is 0 for ranks beyond n_chunks)."""
+    if not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    b = n_chunks * rank // world
+    e = n_chunks * (rank + 1) // world
+    return b, e - b
+
+
+def allgather_rows(local: torch.Tensor, counts, group=None) -> torch.Tensor:
+    """Concatenate every rank's row block (rank order): local is [counts[rank]][...];
+    blocks are padded to the largest count for the collective and trimmed after."""
+    import torch.distributed as dist
+    if not dist.is_initialized() or dist.get_world_size(group) == 1:
+        return local
+    world = dist.get_world_size(group)
+    if len(counts) != world:
+        raise ValueError("one row count per rank")
+    most = max(counts)
+    rest = tuple(local.shape[1:])
+    pad = torch.zeros((most,) + rest, dtype=local.dtype, device=local.device)
+    pad[:local.shape[0]].copy_(local)
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad, group=group)
+    return torch.cat([p[:n] for p, n in zip(parts, counts)])
 
 
 def allreduce_sum_(tensors, group=None) -> None:

@@ -32,21 +32,25 @@ class DustError(RuntimeError):
 
 class _Noise(C.Structure):
     _fields_ = [("seed", C.c_uint32), ("layer", C.c_uint32), ("draw_begin", C.c_uint32),
-                ("draw_count", C.c_uint32), ("K_total", C.c_uint32), ("sigma", C.c_float)]
+                ("draw_count", C.c_uint32), ("K_total", C.c_uint32), ("sigma", C.c_float),
+                ("token_begin", C.c_uint32)]
 
 
 @dataclass(frozen=True)
 class Noise:
-    """Which draws of which layer a call handles (dust_noise)."""
+    """Which draws of which layer a call handles, and the global index of its
+    first token (dust_noise)."""
     seed: int
     layer: int
     draw_begin: int
     draw_count: int
     K_total: int
     sigma: float
+    token_begin: int = 0
 
     def c(self) -> _Noise:
-        return _Noise(self.seed, self.layer, self.draw_begin, self.draw_count, self.K_total, self.sigma)
+        return _Noise(self.seed, self.layer, self.draw_begin, self.draw_count, self.K_total, self.sigma,
+                      self.token_begin)
 
 
 _lib = None
@@ -68,13 +72,14 @@ _SIGS = {
     "dust_layer_estimate_weight_grad": ([_vp, _i, _i, _i, _vp, _i, _f, _Noise, _vp, _i, _vp, _i, _vp, _vp, _sz, _vp],
                                         _i),
     "dust_layer_estimate_weight_grad_workspace": ([_i, _i, _i, _i, _i, _f], _sz),
-    "dust_weight_grad": ([_vp, _vp, _i, _i, _i, _i, _vp, _i, _vp, _sz, _vp], _i),
-    "dust_weight_grad_workspace": ([_i, _i, _i, _i], _sz),
+    "dust_weight_grad": ([_vp, _i, _vp, _i, _i, _i, _i, _vp, _i, _vp, _sz, _vp], _i),
+    "dust_weight_grad_workspace": ([_i, _i, _i, _i, _i], _sz),
     "dust_logits": ([_vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp], _i),
     "dust_logits_workspace": ([_i, _i, _i, _i], _sz),
     "dust_head_row_stats": ([_vp, _vp, _i, _i, _vp, _vp, _vp], _i),
-    "dust_head_step": ([_vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _Noise, _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp], _i),
-    "dust_head_step_workspace": ([_i, _i, _i, _i, _i, _i], _sz),
+    "dust_head_step": ([_vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _Noise, _vp, _vp, _vp, _vp, _i, _vp, _sz,
+                        _vp], _i),
+    "dust_head_step_workspace": ([_i, _i, _i, _i, _i, _i, _i, _i], _sz),
     "dust_head_bp_grad": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp], _i),
     "dust_head_bp_grad_workspace": ([_i, _i, _i, _i], _sz),
     "dust_cosine": ([_vp, _vp, C.c_longlong, _vp, _vp, _sz, _vp], _i),
@@ -85,8 +90,8 @@ _SIGS = {
     "dust_toy_suffix_losses": ([_vp, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp, _Noise, _vp, _vp,
                                 _vp, _sz, _vp], _i),
     "dust_toy_suffix_workspace": ([_i, _i, _i, _i, _i], _sz),
-    "dust_attention_internal_costs": ([_vp, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _vp, _Noise, _vp, _vp, _sz,
-                                       _vp], _i),
+    "dust_attention_internal_costs": ([_vp, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _Noise, _vp,
+                                       _vp, _sz, _vp], _i),
     "dust_attention_internal_costs_workspace": ([_i, _i, _i, _i], _sz),
 }
 
@@ -150,7 +155,10 @@ def workspace(nbytes: int, device=None) -> torch.Tensor:
     key = (dev, torch.cuda.current_stream(dev).cuda_stream)
     cur = _ws.get(key)
     if cur is None or cur.numel() < nbytes:
-        cur = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=dev)
+        new = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=dev)
+        if cur is not None:
+            new[:256].copy_(cur[:256])     # keep a status word that earlier calls may have set
+        cur = new
         _ws[key] = cur
     return cur
 
@@ -164,6 +172,24 @@ def check_offsets(seq_offsets, T: int) -> None:
 
 def poll_status(ws: torch.Tensor) -> None:
     _check(lib().dust_poll_status(_dev(ws, "ws"), _stream()))
+
+
+def poll_all(device=None) -> str:
+    """dust_poll_status on every cached workspace of `device` (default: the
+    current one), each on the stream it serves.  Raises DustError with
+    DUST_ERR_TIMEOUT when a kernel's bounded wait ran out since the last poll
+    (the word is cleared); returns "ok" otherwise."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    failed = None
+    for (d, stream), ws in list(_ws.items()):
+        if d != dev:
+            continue
+        st = lib().dust_poll_status(ws.data_ptr(), stream)
+        if st != 0 and failed is None:
+            failed = DustError(st, lib().dust_last_error().decode())
+    if failed is not None:
+        raise failed
+    return "ok"
 
 
 def selftest_bounded_wait(ws: torch.Tensor, polls: int = 4096) -> None:
@@ -269,15 +295,16 @@ def layer_estimate_noalloc(c: torch.Tensor, seq_offsets, gamma: float, noise: No
 
 # ------------------------------------------------------------------ a6
 def weight_grad(g_hat: torch.Tensor, X: torch.Tensor, G_W: torch.Tensor | None = None, accumulate: bool = False):
+    """G_W [d_out][d_in] fp32 = g_hat^T X; g_hat and X each fp32 or bf16 (they may differ)."""
     T, d_out = g_hat.shape
     d_in = X.shape[1]
-    if X.shape[0] != T or X.dtype != g_hat.dtype:
-        raise ValueError("g_hat and X must share T and dtype")
-    dt = _dtype_code(X)
+    if X.shape[0] != T:
+        raise ValueError("g_hat and X must share T")
+    g_dt, x_dt = _dtype_code(g_hat), _dtype_code(X)
     if G_W is None:
         G_W = torch.empty(d_out, d_in, dtype=torch.float32, device=X.device)
-    ws = workspace(lib().dust_weight_grad_workspace(T, d_in, d_out, dt), X.device)
-    _check(lib().dust_weight_grad(_dev(g_hat, "g_hat"), _dev(X, "X"), dt, T, d_in, d_out,
+    ws = workspace(lib().dust_weight_grad_workspace(T, d_in, d_out, g_dt, x_dt), X.device)
+    _check(lib().dust_weight_grad(_dev(g_hat, "g_hat"), g_dt, _dev(X, "X"), x_dt, T, d_in, d_out,
                                   _dev(G_W, "G_W", torch.float32), int(bool(accumulate)), ws.data_ptr(),
                                   ws.numel(), _stream()))
     return G_W
@@ -312,8 +339,11 @@ def head_step(targets: torch.Tensor, Vc: int, noise: Noise, *, Z: torch.Tensor |
               X: torch.Tensor | None = None, W: torch.Tensor | None = None, V: int | None = None,
               want_c: bool = False, want_bf16: bool = False, want_G_W: bool = False,
               g_hat: torch.Tensor | None = None, g_hat_bf16: torch.Tensor | None = None,
-              accumulate: bool = False):
-    """Returns dict with g_hat, and c / g_hat_bf16 / G_W when requested."""
+              accumulate: bool = False, chunk_begin: int = 0, chunk_count: int | None = None):
+    """Returns dict with g_hat, and c / g_hat_bf16 / G_W when requested.  The
+    chunk range [chunk_begin, chunk_begin + chunk_count) (default: every chunk)
+    sets the outputs' vocabulary columns / rows: g_hat [T][chunk_count Vc],
+    c [chunk_count][draw_count][T], G_W [chunk_count Vc][d_in]."""
     T = targets.numel()
     dev = targets.device
     if Z is not None:
@@ -322,22 +352,25 @@ def head_step(targets: torch.Tensor, Vc: int, noise: Noise, *, Z: torch.Tensor |
         V = W.shape[0]
     if V is None:
         raise ValueError("need Z or W")
+    if chunk_count is None:
+        chunk_count = V // Vc - chunk_begin
+    Vr = chunk_count * Vc
     ref = X if X is not None else W
     dt = _dtype_code(ref) if ref is not None else F32
     d_in = X.shape[1] if X is not None else (W.shape[1] if W is not None else 0)
     if g_hat is None:
-        g_hat = torch.empty(T, V, dtype=torch.float32, device=dev)
-    c = torch.empty(V // Vc, noise.draw_count, T, dtype=torch.float32, device=dev) if want_c else None
+        g_hat = torch.empty(T, Vr, dtype=torch.float32, device=dev)
+    c = torch.empty(chunk_count, noise.draw_count, T, dtype=torch.float32, device=dev) if want_c else None
     g16 = g_hat_bf16
     if g16 is None and want_bf16:
-        g16 = torch.empty(T, V, dtype=torch.bfloat16, device=dev)
-    G_W = torch.empty(V, d_in, dtype=torch.float32, device=dev) if want_G_W else None
-    need = lib().dust_head_step_workspace(T, d_in, V, dt, int(Z is not None), int(want_G_W))
+        g16 = torch.empty(T, Vr, dtype=torch.bfloat16, device=dev)
+    G_W = torch.empty(Vr, d_in, dtype=torch.float32, device=dev) if want_G_W else None
+    need = lib().dust_head_step_workspace(T, d_in, V, Vc, chunk_count, dt, int(Z is not None), int(want_G_W))
     ws = workspace(need, dev)
     _check(lib().dust_head_step(_opt(X, "X"), _opt(W, "W"), dt, _opt(Z, "Z", torch.float32),
-                                _dev(targets, "targets", torch.int32), T, d_in, V, Vc, noise.c(), _opt(c, "c"),
-                                _dev(g_hat, "g_hat", torch.float32), _opt(g16, "g_hat_bf16"), _opt(G_W, "G_W"),
-                                int(bool(accumulate)), ws.data_ptr(), ws.numel(), _stream()))
+                                _dev(targets, "targets", torch.int32), T, d_in, V, Vc, chunk_begin, chunk_count,
+                                noise.c(), _opt(c, "c"), _dev(g_hat, "g_hat", torch.float32), _opt(g16, "g_hat_bf16"),
+                                _opt(G_W, "G_W"), int(bool(accumulate)), ws.data_ptr(), ws.numel(), _stream()))
     return {"g_hat": g_hat, "c": c, "g_hat_bf16": g16, "G_W": G_W}
 
 
@@ -409,9 +442,10 @@ def toy_suffix_losses(Y, seq_offsets, Wq, Wk, Wv, Wo, Wout, targets, noise: Nois
     return loss, c
 
 
-def attention_internal_costs(Y, seq_offsets, Wq, Wk, Wv, Wo, which: int, G, noise: Noise):
-    """Costs of the draws of projection `which` (0 q, 1 k, 2 v) scored through the
-    attention output against its estimated error G: c [draw_count][T]."""
+def attention_internal_costs(Y, seq_offsets, Wq, Wk, Wv, Wo, which: int, G, noise: Noise, Wg=None, E=None):
+    """Costs of the draws of `which` (0 q, 1 k, 2 v, 3 the gate's pre-activation,
+    4 the value embedding) scored through the attention output against its
+    estimated error G; the values are Y Wv^T + s(Y Wg^T) E: c [draw_count][T]."""
     T, d = Y.shape
     dh = Wq.shape[0]
     c = torch.empty(noise.draw_count, T, dtype=torch.float32, device=Y.device)
@@ -419,7 +453,7 @@ def attention_internal_costs(Y, seq_offsets, Wq, Wk, Wv, Wo, which: int, G, nois
     f32 = torch.float32
     _check(lib().dust_attention_internal_costs(_dev(Y, "Y", f32), T, d, _dev(seq_offsets, "seq_offsets", torch.int32),
                                                seq_offsets.numel() - 1, _dev(Wq, "Wq", f32), _dev(Wk, "Wk", f32),
-                                               _dev(Wv, "Wv", f32), _dev(Wo, "Wo", f32), dh, int(which),
-                                               _dev(G, "G", f32), noise.c(), c.data_ptr(), ws.data_ptr(), ws.numel(),
-                                               _stream()))
+                                               _dev(Wv, "Wv", f32), _dev(Wo, "Wo", f32), _opt(Wg, "Wg", f32),
+                                               _opt(E, "E", f32), dh, int(which), _dev(G, "G", f32), noise.c(),
+                                               c.data_ptr(), ws.data_ptr(), ws.numel(), _stream()))
     return c

@@ -13,9 +13,17 @@ the head's G_W (a6).  The synthetic costs c that stand in for the perturbed
 forward of the hidden layers are produced once, before timing (harness).
 
 Metric: draws x tokens per second summed over the layers of one step,
-value = sum_layers K * T * N_ranks / max-over-ranks step time.  Every rank
-processes its own batch (weak scaling, data parallel); with N > 1 the weight
-estimates are summed over ranks by one NCCL all-reduce per step.
+value = the draws x tokens of all ranks / max-over-ranks step time.  With
+N > 1 GPUs the step is split one of three ways (--shard):
+  sequences (default): every rank processes its own batch of whole sequences
+    (weak scaling, data parallel), its tokens placed after the previous
+    ranks' in the global batch (noise token_begin); the weight estimates are
+    summed over ranks by one NCCL all-reduce per step;
+  draws: every rank runs a range of the K draws of the same batch (strong
+    scaling); the partial weight estimates are summed by the all-reduce;
+  vocab: the hidden layers as in `draws`, the LM head split by vocabulary
+    chunk (each rank all K draws of a range of chunk passes); its disjoint
+    G_W rows are gathered (strong scaling).
 
 Prints one JSON line (rank 0).
 """
@@ -76,6 +84,8 @@ def parse_args():
     p.add_argument("--draws", type=int, default=0, help="override the workload's K")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--shard", choices=["sequences", "draws", "vocab"], default="sequences",
+                   help="how N > 1 ranks split the step (see above); at N = 1 every split is the whole step")
     p.add_argument("--fused", action="store_true",
                    help="hidden layers with d_in a multiple of 64 up to 512 run the draw reduction and the weight "
                         "estimate as one kernel (dust_layer_estimate_weight_grad)")
@@ -184,22 +194,30 @@ def max_over_ranks(x, world):
 
 # ------------------------------------------------------------------ the step
 class Step:
-    """Device-resident buffers and the sequence of C-ABI calls of one step."""
+    """Device-resident buffers and the sequence of C-ABI calls of one step on
+    this rank: its sequences (shard 'sequences'), its draws ('draws') or, for
+    the head, its vocabulary chunks ('vocab')."""
 
-    def __init__(self, w: I.Workload, K: int, rank: int, world: int, fused: bool = False):
+    def __init__(self, w: I.Workload, K: int, rank: int, world: int, fused: bool = False, shard: str = "sequences"):
         import torch
-        from activation_perturbation_es_b200 import dust
-        self.torch, self.dust, self.w, self.K, self.world = torch, dust, w, K, world
+        from activation_perturbation_es_b200 import dust, dp
+        self.torch, self.dust, self.dp, self.w, self.K, self.world = torch, dust, dp, w, K, world
+        self.shard = shard
         dev = torch.device("cuda", torch.cuda.current_device())
         self.dev = dev
         bf = torch.bfloat16
         T = w.T
+        by_seq = self.shard == "sequences"
+        data_off = rank * 7919 if by_seq else 0          # each rank's own batch, or one batch for all
+        tok0 = rank * T if by_seq else 0                 # global index of this rank's first token
+        d0, nd = (0, K) if by_seq else dp.draw_range(K, world, rank)
+        self.draws = nd
         self.off = torch.from_numpy(I.uniform_offsets(w.n_seq, w.seq_len)).to(dev)
         self.hidden = []
         self.host = {}          # pinned host copies of every per-step input (for e2e)
         for hl in w.hidden:
-            li = I.layer_inputs(w, hl, seed_offset=rank * 7919)
-            nz = dust.Noise(w.seed + rank, hl.layer, 0, K, K, w.sigma)
+            li = I.layer_inputs(w, hl, seed_offset=data_off)
+            nz = dust.Noise(w.seed, hl.layer, d0, nd, K, w.sigma, token_begin=tok0)
             u = torch.from_numpy(li["u"]).to(dev)
             c = dust.synth_costs(u, nz, w.eps_scale)          # harness: stands in for the perturbed forward
             del u
@@ -213,15 +231,28 @@ class Step:
             self.hidden.append(L)
         self.head = None
         if w.V:
-            hi = I.head_inputs(w, seed_offset=rank * 7919)
-            nz = dust.Noise(w.seed + rank, w.head_layer, 0, K, K, w.sigma)
+            hi = I.head_inputs(w, seed_offset=data_off)
+            W = I.head_inputs(w)["W"]                        # the head's weights are shared by all ranks
+            n_chunks = w.V // w.Vc
+            if self.shard == "vocab":
+                cb, cc = dp.chunk_range(n_chunks, world, rank)
+                hd0, hnd = 0, K
+            else:
+                cb, cc = 0, n_chunks
+                hd0, hnd = d0, nd
+            Vr = cc * w.Vc
+            nz = dust.Noise(w.seed, w.head_layer, hd0, hnd, K, w.sigma, token_begin=tok0)
             self.head = {"nz": nz, "X": torch.from_numpy(hi["X"]).to(dev, bf),
-                         "W": torch.from_numpy(hi["W"]).to(dev, bf),
+                         "W": torch.from_numpy(W).to(dev, bf),
                          "y": torch.from_numpy(hi["y"]).to(dev),
+                         "chunks": (cb, cc), "rows": [dp.chunk_range(n_chunks, world, r)[1] * w.Vc
+                                                      for r in range(world)] if self.shard == "vocab" else None,
                          "Z": torch.empty(T, w.V, dtype=torch.float32, device=dev),
-                         "g": torch.empty(T, w.V, dtype=torch.float32, device=dev),
-                         "g16": torch.empty(T, w.V, dtype=bf, device=dev),
-                         "G": torch.empty(w.V, w.head_d, dtype=torch.float32, device=dev)}
+                         "g": torch.empty(T, max(Vr, 1), dtype=torch.float32, device=dev),
+                         "g16": torch.empty(T, max(Vr, 1), dtype=bf, device=dev),
+                         "G": torch.empty(max(Vr, 1), w.head_d, dtype=torch.float32, device=dev)}
+            self.head["draws"] = hnd
+            self.head["Vr"] = Vr
         torch.cuda.synchronize()
         self.stage_names = []
         for L in self.hidden:
@@ -231,9 +262,28 @@ class Step:
         if self.head:
             self.stage_names += ["head:logits", "head:ce_estimate", "head:weight_grad"]
         self.events = None
+        self.G_head_all = None
 
     def units(self):
-        return self.K * self.w.T * (len(self.hidden) + (1 if self.head else 0))
+        """Draws x tokens of one step summed over the layers, on this rank."""
+        u = self.draws * self.w.T * len(self.hidden)
+        if self.head:
+            # a vocabulary-chunk shard runs all K draws on a fraction Vr/V of the head's chunks
+            u += self.head["draws"] * self.w.T * self.head["Vr"] / self.w.V
+        return u
+
+    def total_units(self):
+        """Draws x tokens of one step over all ranks: every rank's own batch
+        (sequences), or the one batch's K draws of every layer (draws, vocab)."""
+        per_batch = self.K * self.w.T * (len(self.hidden) + (1 if self.head else 0))
+        return per_batch * self.world if self.shard == "sequences" else per_batch
+
+    def scaling(self):
+        return "weak" if self.shard == "sequences" else "strong"
+
+    def parallelism(self):
+        return {"sequences": f"dp{self.world}", "draws": f"draws{self.world}",
+                "vocab": f"draws{self.world}+head_vocab{self.world}"}[self.shard]
 
     def make_events(self, n_steps):
         ev = self.torch.cuda.Event
@@ -264,10 +314,10 @@ class Step:
             mark()
             dust.logits(H["X"], H["W"], Z=H["Z"])
             mark()
-            # row statistics + all chunk passes (a3 + a5) on the cached logits of a2
-            dust.head_step(H["y"], self.w.Vc, H["nz"], Z=H["Z"], g_hat=H["g"], g_hat_bf16=H["g16"])
+            self._head(H)
             mark()
-            dust.weight_grad(H["g16"], H["X"], G_W=H["G"])
+            if H["Vr"]:
+                dust.weight_grad(H["g16"], H["X"], G_W=H["G"])
         mark()
         if self.world > 1:
             self.allreduce()
@@ -287,10 +337,18 @@ class Step:
             H = self.head
             cur.wait_event(ready[j])
             dust.logits(H["X"], H["W"], Z=H["Z"])
-            dust.head_step(H["y"], self.w.Vc, H["nz"], Z=H["Z"], g_hat=H["g"], g_hat_bf16=H["g16"])
-            dust.weight_grad(H["g16"], H["X"], G_W=H["G"])
+            self._head(H)
+            if H["Vr"]:
+                dust.weight_grad(H["g16"], H["X"], G_W=H["G"])
         if self.world > 1:
             self.allreduce()
+
+    def _head(self, H):
+        """Row statistics + this rank's chunk passes (a3 + a5) on the cached logits of a2."""
+        cb, cc = H["chunks"]
+        if cc:
+            self.dust.head_step(H["y"], self.w.Vc, H["nz"], Z=H["Z"], g_hat=H["g"], g_hat_bf16=H["g16"],
+                                chunk_begin=cb, chunk_count=cc)
 
     def _estimate(self, L):
         """The draw reduction; fused with the weight estimate when L is eligible."""
@@ -303,8 +361,14 @@ class Step:
                                      g_hat_bf16=L["g16"])
 
     def allreduce(self):
-        from activation_perturbation_es_b200 import dp
-        dp.allreduce_sum_([L["G"] for L in self.hidden] + ([self.head["G"]] if self.head else []))
+        """The step's exchange: the weight estimates summed over ranks; with the
+        head split by vocabulary chunk, its disjoint G_W rows gathered instead."""
+        dp = self.dp
+        by_vocab = self.head is not None and self.head["rows"] is not None
+        dp.allreduce_sum_([L["G"] for L in self.hidden] + ([self.head["G"]] if self.head and not by_vocab else []))
+        if by_vocab:
+            H = self.head
+            self.G_head_all = dp.allgather_rows(H["G"][:H["Vr"]], H["rows"])
 
     def stage_times(self, n_steps):
         """Mean ms per stage over the timed steps."""
@@ -325,7 +389,7 @@ def main():
     w = I.WORKLOADS[args.workload]
     K = args.draws or w.K
     peaks = load_peaks()
-    step = Step(w, K, rank, world, fused=args.fused)
+    step = Step(w, K, rank, world, fused=args.fused, shard=args.shard)
     for _ in range(args.warmup):
         step.run()
     torch.cuda.synchronize()
@@ -345,27 +409,35 @@ def main():
         barrier(world)
     ms_total = max_over_ranks(t0.elapsed_time(t1), world)
     ms_step = ms_total / args.steps
-    value = step.units() * world / (ms_step / 1e3)
+    value = step.total_units() / (ms_step / 1e3)
     stages = step.stage_times(args.steps)
     clocks = clk.summary()
 
     kernels = kernel_report(step, stages, peaks, clocks)
-    dominant = max(kernels, key=lambda k: k["ms"])
+    dominant = max((k for k in kernels if not k.get("idle")), key=lambda k: k["ms"])
     e2e = None if args.no_e2e else e2e_run(step, args, world)
+    # every tcgen05 / fused kernel records a run-out bounded wait in its workspace's status word:
+    # read them all back, so that an aborted kernel cannot pass for a fast one
+    from activation_perturbation_es_b200 import dust
+    try:
+        status = dust.poll_all()
+    except dust.DustError as e:
+        status = f"error: {e}"
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, K)
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": step.scaling(),
             "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded; inputs > L2, no flush needed)",
             "config": {"workload": w.name, "tokens_per_rank": w.T, "n_seq": w.n_seq, "seq_len": w.seq_len,
                        "draws": K, "sigma": w.sigma, "gamma_hidden": w.gamma,
                        "hidden": [[h.d_in, h.d_out] for h in w.hidden],
                        "head": {"d": w.head_d, "V": w.V, "Vc": w.Vc} if w.V else None,
-                       "parallelism": f"dp{world}", "l2": "inputs larger than L2 (126 MB); no flush",
+                       "parallelism": step.parallelism(), "shard": step.shard,
+                       "l2": "inputs larger than L2 (126 MB); no flush",
                        "fused_estimate_wgrad": bool(args.fused),
                        "arithmetic": "f32 noise, cross entropy and reductions; bf16 GEMM operands with f32 "
                                      "accumulation in TMEM (tcgen05)"},
@@ -377,11 +449,14 @@ def main():
             "e2e": e2e,
             "gpu_launches": launches_per_step(step) * args.steps,
             "clocks": clocks,
+            "status": status,
         }
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+    if status != "ok":
+        sys.exit(f"bench: device status word set ({status}): the timed kernels did not all complete")
 
 
 def launches_per_step(step):
@@ -393,18 +468,22 @@ def launches_per_step(step):
             n += 2                               # fused reduction + weight GEMM, split reduction
             continue
         n += 1                                   # draw reduction
-        n += 1 if step.dust.lib().dust_weight_grad_workspace(step.w.T, L["hl"].d_in, L["hl"].d_out, 1) <= 256 else 2
+        n += 1 if step.dust.lib().dust_weight_grad_workspace(step.w.T, L["hl"].d_in, L["hl"].d_out, 1, 1) <= 256 else 2
     if step.head:
         n += 1                                   # logits GEMM
-        n += 2                                   # row stats + chunk passes
-        n += 1 if step.dust.lib().dust_weight_grad_workspace(step.w.T, step.w.head_d, step.w.V, 1) <= 256 else 2
+        Vr = step.head["Vr"]
+        if Vr:
+            n += 2                               # row stats + chunk passes
+            n += 1 if step.dust.lib().dust_weight_grad_workspace(step.w.T, step.w.head_d, Vr, 1, 1) <= 256 else 2
     return n
 
 
 def load_traffic():
-    """ncu DRAM bytes per output unit from profiles/traffic.txt, for kernels whose
+    """ncu DRAM bytes per unit from profiles/traffic.txt, for kernels whose
     source files ('+'-joined, hashed in order) are unchanged since the capture
-    (sha1 prefix match); else absent."""
+    (sha1 prefix match); else absent.  A kernel may have several lines, one per
+    unit its traffic grows with (e.g. r per draw x token, g per token x
+    channel); returns {kernel: [(bytes_per_unit, unit), ...]}."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     out = {}
@@ -422,12 +501,21 @@ def load_traffic():
             continue
         cur = h.hexdigest()[:len(sha)]
         if cur == sha:
-            out[kernel] = (float(per_unit), unit)
+            out.setdefault(kernel, []).append((float(per_unit), unit))
     return out
 
 
+def traffic_bytes(terms, K, T, d_out):
+    """Per-launch DRAM bytes from per-unit terms (None when a term's unit is unknown)."""
+    counts = {"draw_x_token": float(K) * T, "token_x_out_channel": float(T) * d_out,
+              "token_x_vocab": float(T) * d_out}
+    if not terms or any(u not in counts for _, u in terms):
+        return None
+    return sum(b * counts[u] for b, u in terms)
+
+
 def kernel_report(step, stages, peaks, clocks):
-    w, K, T = step.w, step.K, step.w.T
+    w, T = step.w, step.w.T
     f_peak = peaks["sm_max_mhz"]
     alu_peak = 148 * LANES_PER_SM * f_peak * 1e6 / 1e12          # T lane-slots/s
     out = []
@@ -436,11 +524,16 @@ def kernel_report(step, stages, peaks, clocks):
     for name, ms in zip(names, stages):
         layer, kind = name.split(":")
         rec = {"name": name, "ms": float(ms)}
+        # this rank's share: its draws, and for the head its vocabulary range
         if layer == "head":
-            d_in, d_out = w.head_d, w.V
+            d_in, d_out, K = w.head_d, (w.V if kind == "logits" else step.head["Vr"]), step.head["draws"]
         else:
             hl = next(h for h in w.hidden if h.name == layer)
-            d_in, d_out = hl.d_in, hl.d_out
+            d_in, d_out, K = hl.d_in, hl.d_out, step.draws
+        if d_out == 0 or ms <= 0:
+            rec["idle"] = True                   # a rank with no head chunks
+            out.append(rec)
+            continue
         if kind == "scan":
             byts = 8.0 * K * T
             ach = byts / (ms / 1e3) / 1e9
@@ -467,11 +560,16 @@ def kernel_report(step, stages, peaks, clocks):
             slots = float(K) * T * d_out * slots_el
             ach = slots / (ms / 1e3) / 1e12
             tkey = "head_chunk_kernel" if layer == "head" else "layer_estimate"
-            tr = traffic.get(tkey)
+            tr = traffic_bytes(traffic.get(tkey), K, T, d_out)
+            # the bytes the step must move: the head reads Z (4 B per logit) and writes g in fp32 and bf16
+            # (6 B); the reduction reads r (4 B per draw x token) and writes g in fp32 and bf16
+            alg_bytes = 10.0 * T * d_out if layer == "head" else 4.0 * K * T + 6.0 * T * d_out
             rec |= {"bound": "alu", "achieved": ach, "peak": alu_peak, "unit": "T lane-slots/s",
-                    "frac": ach / alu_peak, "traffic": tr[0] * T * d_out if tr else None,
-                    "traffic_source": "profiles/traffic.txt (ncu small case, scaled by tokens x channels)"
+                    "frac": ach / alu_peak, "traffic": tr,
+                    "traffic_source": "profiles/traffic.txt (ncu capture, each term scaled by its own unit count)"
                     if tr else None,
+                    "algorithmic_bytes": alg_bytes,
+                    "traffic_over_algorithmic": tr / alg_bytes if tr else None,
                     "algorithmic_slots": slots,
                     "slots_per_element": slots_el, "clock_mhz_for_peak": f_peak,
                     "gaussians_per_s": float(K) * T * d_out / (ms / 1e3),
@@ -528,7 +626,7 @@ def e2e_run(step, args, world):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(t0.elapsed_time(t1), world) / n
-    return {"value": step.units() * world / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+    return {"value": step.total_units() / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": n,
             "copies": "pinned host -> device on a copy stream, overlapped with the previous layer's compute"}
 

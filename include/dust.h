@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define DUST_ABI_VERSION 1
+#define DUST_ABI_VERSION 2
 
 typedef enum {
     DUST_OK = 0,
@@ -61,11 +61,16 @@ typedef enum {
 
 typedef enum { DUST_F32 = 0, DUST_BF16 = 1 } dust_dtype;
 
-/* Which draws of which layer a call handles.  The noise element of draw i,
- * token t, channel j is a(seed, layer, i, t, j); a call handles the global
- * draws [draw_begin, draw_begin + draw_count) and scales by the whole
- * population K_total, so that splitting the draws of one estimate over several
- * calls (accumulate = 1) gives the same sum [CA, error equation]. */
+/* Which draws of which layer a call handles, and where its tokens sit in the
+ * global batch.  The noise element of draw i, token t (row t of the call's
+ * tensors), channel j is a(seed, layer, i, token_begin + t, j).  A call
+ * handles the global draws [draw_begin, draw_begin + draw_count) and scales by
+ * the whole population K_total, so that splitting the draws of one estimate
+ * over several calls (accumulate = 1) gives the same sum [CA, error equation];
+ * token_begin is the global index of the call's first token, so that a batch
+ * split by whole sequences over several calls or ranks draws, token for
+ * token, the noise of one call over the whole batch ([CA]: a_t is drawn per
+ * token). */
 typedef struct {
     uint32_t seed;        /* Philox key word 0 */
     uint32_t layer;       /* Philox key word 1 (one value per perturbed layer) */
@@ -73,6 +78,7 @@ typedef struct {
     uint32_t draw_count;  /* number of draws handled by this call (> 0) */
     uint32_t K_total;     /* population size K of the 1/(K sigma) scale (> 0) */
     float sigma;          /* noise scale (> 0, finite) */
+    uint32_t token_begin; /* global index of row 0 of the call's tokens (< 2^31) */
 } dust_noise;
 
 /* ------------------------------------------------------------------ status */
@@ -139,21 +145,26 @@ size_t dust_layer_estimate_workspace(int draw_count, int T, int d_out, int is_r,
  * owns all device memory and hands it only the device pointers of its inputs
  * and outputs, or a caller whose memory pool is fully reserved.  The pages
  * have no counterpart: it is a deployment variant of the same computation
- * (reward scan into scratch, then the draw reduction) whose scratch for r is a
- * fixed 16 MiB device array inside the library image instead of a workspace.
+ * (reward scan into scratch, then the draw reduction) whose scratch is a fixed
+ * device array inside the library image instead of a workspace: 16 MiB for
+ * the rewards plus 64 KiB for the chunk maps of the chunked scan.
  *   c: [draw_count][T] fp32 costs; other arguments as dust_layer_estimate.
+ *   The scan takes dust_layer_estimate's path (per sequence, or over
+ *   1024-token chunks for few long sequences), so the result is the same bits.
  *   Limit: draw_count * T <= 4194304 when gamma > 0 (DUST_ERR_WORKSPACE
  *   otherwise, nothing launched); split the draws over calls with
  *   accumulate = 1 for more.  gamma = 0 uses no scratch.
- *   The array costs 16 MiB on every GPU that loads the library, until exit.
+ *   The array costs 16.06 MiB on every GPU that loads the library, until exit.
  *   It is shared by all calls: calls whose kernels may overlap on the GPU race
  *   on it and must be serialised by the caller.  It keeps the last call's
  *   contents; nothing needs to start at zero (the scan rewrites every r the
  *   reduction reads).
  *   Set-up: the first call on a device looks the array's device address up
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.  The call allocates nothing (no cudaMalloc,
- *   cudaFree or allocating library routine). */
+ *   (cudaGetSymbolAddress) with that device current and caches it for the
+ *   process; make that first call before any stream capture.  After
+ *   cudaDeviceReset of a device the cached address is stale: do not call this
+ *   entry point on that device again.  The call allocates nothing (no
+ *   cudaMalloc, cudaFree or allocating library routine). */
 dust_status dust_layer_estimate_noalloc(const float *c, int T, int d_out,
                                         const int32_t *seq_offsets, int n_seq, float gamma,
                                         dust_noise nz, float *g_hat, void *g_hat_bf16,
@@ -173,6 +184,11 @@ dust_status dust_layer_estimate_noalloc(const float *c, int T, int d_out,
  *   G_W: [d_out][d_in] fp32, overwritten (accumulate = 0) or added to;
  *   g_hat_out: nullable [T][d_out] fp32, receives g_hat (the same bits as
  *     dust_layer_estimate's g_hat) for checks.
+ *   draw_count: at most 1048576 per call (DUST_ERR_UNSUPPORTED otherwise);
+ *     split larger populations over calls with accumulate = 1.  The kernel's
+ *     waits on a stage's production are bounded by a time budget that grows
+ *     with the draw count (2 s + 20 us per draw), after which it sets the
+ *     status word (DUST_ERR_TIMEOUT from dust_poll_status) and returns.
  * The bf16 g values are those of dust_layer_estimate's g_hat_bf16, so G_W
  * agrees with dust_layer_estimate followed by dust_weight_grad up to the
  * order of the fp32 accumulation.  Token splits are summed in a fixed order.
@@ -188,16 +204,18 @@ size_t dust_layer_estimate_weight_grad_workspace(int draw_count, int T, int d_in
 
 /* ------------------------------------------------------------------ a6: weight
  * [CA, weight equation] G_W[o][i] (+)= sum_t g_hat[t][o] X[t][i].
- * g_hat: [T][d_out], X: [T][d_in], both of dtype `dt` (DUST_BF16 runs on the
- * tcgen05 tensor cores with fp32 accumulation in TMEM and needs d_in and d_out
- * multiples of 16 and pointers 128-byte aligned; DUST_F32 runs on fp32 CUDA
- * cores).  G_W: [d_out][d_in] fp32 (the layout of W).  Split over T with a
- * fixed-order reduction: results do not depend on the launch.
+ * g_hat: [T][d_out] of dtype g_dt, X: [T][d_in] of dtype x_dt.  Both bf16:
+ * the tcgen05 tensor cores with fp32 accumulation in TMEM when d_in and d_out
+ * are multiples of 16 and the pointers 128-byte aligned (else CUDA cores);
+ * both fp32: fp32 CUDA cores; mixed (fp32 g with bf16 X, or bf16 g with fp32
+ * X): CUDA cores, each bf16 element widened to fp32 exactly, fp32 products.
+ * G_W: [d_out][d_in] fp32 (the layout of W).  Split over T with a fixed-order
+ * reduction: results do not depend on the launch.
  * Workspace: dust_weight_grad_workspace(). */
-dust_status dust_weight_grad(const void *g_hat, const void *X, dust_dtype dt,
+dust_status dust_weight_grad(const void *g_hat, dust_dtype g_dt, const void *X, dust_dtype x_dt,
                              int T, int d_in, int d_out, float *G_W, int accumulate,
                              void *ws, size_t ws_bytes, void *stream);
-size_t dust_weight_grad_workspace(int T, int d_in, int d_out, dust_dtype dt);
+size_t dust_weight_grad_workspace(int T, int d_in, int d_out, dust_dtype g_dt, dust_dtype x_dt);
 
 /* ------------------------------------------------------------------ a2: logits
  * Clean head forward Z[t][v] = sum_k X[t][k] W[v][k] (no bias), fp32 out.
@@ -214,7 +232,11 @@ dust_status dust_head_row_stats(const float *Z, const int32_t *targets, int T, i
                                 float *lse, float *ell, void *stream);
 
 /* ------------------------------------------------------------------ a2+a3+a5+a6: head
- * [IS3] LM-head step over all V/Vc vocabulary chunks.  For chunk
+ * [IS3] LM-head step over the vocabulary chunks [chunk_begin, chunk_begin +
+ * chunk_count) of width Vc (all of them: chunk_begin = 0, chunk_count = V/Vc).
+ * The chunk passes are independent given the clean logits, so the chunks can
+ * be split over calls or ranks (head sharding by vocabulary); their g columns
+ * and G_W rows are disjoint.  For chunk
  * [v0, v0 + Vc) and draw i, the logits of the chunk are perturbed,
  * z~ = z + sigma a(i, t, v) for v in the chunk, and the change of the
  * full-vocabulary cross entropy is [CA] c = CE(z~, y) - CE(z, y), computed as
@@ -229,18 +251,25 @@ dust_status dust_head_row_stats(const float *Z, const int32_t *targets, int T, i
  *   Vc: chunk width; must divide V; supported: multiples of 128 up to 1024,
  *      of 256 up to 2048 and of 512 up to 4096 (Vc = V is the reading where
  *      every draw perturbs the whole vocabulary).
- *   c_out: nullable [V/Vc][draw_count][T] fp32, the costs of every pass.
- *   g_hat: [T][V] fp32 (overwritten, or added to when accumulate = 1).
- *   g_hat_bf16: nullable [T][V] bf16 copy of the final g_hat.
- *   G_W: nullable [V][d_in] fp32, overwritten with g_hat^T X (a6) computed
- *      from the final g_hat (requires X).
- * Workspace: dust_head_step_workspace(). */
+ *   chunk_begin, chunk_count: the chunk range (0 <= chunk_begin,
+ *      chunk_count >= 1, chunk_begin + chunk_count <= V/Vc); below,
+ *      Vr = chunk_count Vc and column / row m of the outputs is vocabulary id
+ *      chunk_begin Vc + m.  The statistics lse and the softmax p always cover
+ *      the whole vocabulary.
+ *   c_out: nullable [chunk_count][draw_count][T] fp32, the costs of every pass.
+ *   g_hat: [T][Vr] fp32 (overwritten, or added to when accumulate = 1).
+ *   g_hat_bf16: nullable [T][Vr] bf16 copy of the final g_hat.
+ *   G_W: nullable [Vr][d_in] fp32, overwritten with g_hat^T X (a6) computed
+ *      from the final g_hat (requires X): rows chunk_begin Vc .. + Vr of the
+ *      full head's estimate.
+ * Workspace: dust_head_step_workspace() with the same chunk_count. */
 dust_status dust_head_step(const void *X, const void *W, dust_dtype dt, const float *Z,
                            const int32_t *targets, int T, int d_in, int V, int Vc,
-                           dust_noise nz, float *c_out, float *g_hat, void *g_hat_bf16,
-                           float *G_W, int accumulate, void *ws, size_t ws_bytes,
-                           void *stream);
-size_t dust_head_step_workspace(int T, int d_in, int V, dust_dtype dt, int has_Z, int want_G_W);
+                           int chunk_begin, int chunk_count, dust_noise nz, float *c_out,
+                           float *g_hat, void *g_hat_bf16, float *G_W, int accumulate,
+                           void *ws, size_t ws_bytes, void *stream);
+size_t dust_head_step_workspace(int T, int d_in, int V, int Vc, int chunk_count, dust_dtype dt,
+                                int has_Z, int want_G_W);
 
 /* ------------------------------------------------------------------ cosine tuner
  * cnblogs Dust explainer, section "真正的工作量：压住干扰" (last paragraph): the
@@ -301,23 +330,35 @@ dust_status dust_toy_suffix_losses(const float *Y, int T, int d, const int32_t *
 size_t dust_toy_suffix_workspace(int draw_count, int T, int d, int dh, int V);
 
 /* Attention-internal scoring (cnblogs Dust explainer, section
- * "真正的工作量：压住干扰", second measure): the draws of one internal
- * projection of a causal softmax attention head (which: 0 = q, 1 = k,
- * 2 = v; noise channel = projection channel, dh wide) are scored through the
- * attention output z = Attn(q, k, v) Wo^T against its estimated error G:
+ * "真正的工作量：压住干扰", second measure): the draws of one internal quantity
+ * of a causal softmax attention head (query, key, value, gate, value
+ * embedding; noise channel = that quantity's channel, dh wide) are scored
+ * through the attention output z = Attn(q, k, v) Wo^T against its estimated
+ * error G:
  *   c[k][t] = -< z~_t - z_t, G_t >   (first order: the loss change l~ - l),
  * computed as -< o~_t - o_t, G_t Wo > since z is linear in the attention's
- * value output o.  q, k, v = Y Wq^T, Y Wk^T, Y Wv^T (scores / sqrt(dh)),
- * one head per sequence.  Y, G: [T][d]; Wq, Wk, Wv: [dh][d]; Wo: [d][dh];
+ * value output o.  q, k = Y Wq^T, Y Wk^T (scores / sqrt(dh)), one head per
+ * sequence.  The values carry each token's value embedding through a gate:
+ *   v_t = Y_t Wv^T + s(Y_t Wg^T) * E_t   (s = logistic sigmoid per channel;
+ *                                         s = 1 when Wg is NULL; E NULL: no
+ *                                         embedding, v = Y Wv^T).
+ * The library's reading of the pages, which name the gate and the value
+ * embedding among the attention's internals and say both are read by later
+ * tokens (credit-assignment section): both act on the values.
+ *   which: 0 = q, 1 = k, 2 = v (the noise is added to the projection),
+ *          3 = the gate's pre-activation Y Wg^T (needs Wg and E),
+ *          4 = the value embedding E (needs E).
+ * Y, G: [T][d]; Wq, Wk, Wv, Wg: [dh][d]; Wo: [d][dh]; E: [T][dh];
  * c: [draw_count][T].  The costs feed dust_layer_estimate with d_out = dh
- * (the pages give keys and values a discount gamma close to 1).
- * Supported: dh % 4 == 0, dh <= 128.  fp32 CUDA cores.
+ * (the pages give keys, values, gates and value embeddings a discount gamma
+ * close to 1).  Supported: dh % 4 == 0, dh <= 128.  fp32 CUDA cores.
  * Workspace: dust_attention_internal_costs_workspace(). */
 dust_status dust_attention_internal_costs(const float *Y, int T, int d, const int32_t *seq_offsets,
                                           int n_seq, const float *Wq, const float *Wk,
-                                          const float *Wv, const float *Wo, int dh, int which,
-                                          const float *G, dust_noise nz, float *c, void *ws,
-                                          size_t ws_bytes, void *stream);
+                                          const float *Wv, const float *Wo, const float *Wg,
+                                          const float *E, int dh, int which, const float *G,
+                                          dust_noise nz, float *c, void *ws, size_t ws_bytes,
+                                          void *stream);
 size_t dust_attention_internal_costs_workspace(int draw_count, int T, int d, int dh);
 
 #ifdef __cplusplus

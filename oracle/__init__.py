@@ -55,7 +55,7 @@ def lib():
         L.orc_reward_scan_brute.argtypes = [_f32p, _f64p, i32, i32, _i32p, i32, dbl]
         L.orc_reward_scan_brute.restype = i32
         L.orc_layer_estimate.argtypes = [_f32p, i32, i32, i32, i32, _i32p, i32, dbl,
-                                         u32, u32, u32, i32, dbl, _i32p, i32,
+                                         u32, u32, u32, u32, i32, dbl, _i32p, i32,
                                          _nullable(_i32p), i32, _f64p]
         L.orc_layer_estimate.restype = i32
         L.orc_weight_grad.argtypes = [_f32p, _f32p, i32, i32, i32, _i32p, i32, _f64p]
@@ -77,7 +77,8 @@ def lib():
                                             _f32p, _f32p, _f32p, _f32p, i32, _f32p, i32,
                                             _i32p, u32, u32, dbl, i32, _i32p, i32, _f64p]
         L.orc_toy_suffix_losses.restype = i32
-        L.orc_attention_internal_costs.argtypes = [_f32p, i32, i32, _i32p, i32, _f32p, _f32p, _f32p, _f32p, i32, i32,
+        L.orc_attention_internal_costs.argtypes = [_f32p, i32, i32, _i32p, i32, _f32p, _f32p, _f32p, _f32p,
+                                                   _nullable(_f32p), _nullable(_f32p), i32, i32,
                                                    _f32p, u32, u32, dbl, _i32p, i32, _f64p]
         L.orc_attention_internal_costs.restype = i32
         _lib = L
@@ -179,8 +180,9 @@ def reward_scan(c, seq_offsets, gamma, brute=False) -> np.ndarray:
 
 
 def layer_estimate(c_or_r, is_r, d_out, seq_offsets, gamma, seed, layer, draw_begin,
-                   K_total, sigma, toks, chans=None) -> np.ndarray:
-    """g[len(toks)][len(chans) or d_out] in float64; c_or_r is [K][T] float32."""
+                   K_total, sigma, toks, chans=None, token_begin=0) -> np.ndarray:
+    """g[len(toks)][len(chans) or d_out] in float64; c_or_r is [K][T] float32;
+    column t draws the noise of global token token_begin + t."""
     a = _f32(c_or_r)
     K, T = a.shape
     off = _i32(seq_offsets)
@@ -189,7 +191,7 @@ def layer_estimate(c_or_r, is_r, d_out, seq_offsets, gamma, seed, layer, draw_be
     nc = d_out if chans is None else len(chans_a)
     g = np.zeros((len(toks), nc), np.float64)
     _check(lib().orc_layer_estimate(a, int(bool(is_r)), K, T, d_out, off, len(off) - 1,
-                                    float(gamma), seed, layer, draw_begin, K_total, float(sigma),
+                                    float(gamma), seed, layer, draw_begin, int(token_begin), K_total, float(sigma),
                                     toks, len(toks), chans_a, nc, g), "layer_estimate")
     return g
 
@@ -288,15 +290,19 @@ def toy_suffix_losses(X, W, seq_offsets, Wq, Wk, Wv, Wo, Wout, targets, seed, la
 
 # ---------------------------------------------------------------- attention-internal scoring
 
-def attention_internal_costs(Y, seq_offsets, Wq, Wk, Wv, Wo, which, G, seed, layer, sigma, draws) -> np.ndarray:
-    """c[n][t] = -<z~_t - z_t, G_t> for perturbations of projection `which` (0 q, 1 k, 2 v)."""
+def attention_internal_costs(Y, seq_offsets, Wq, Wk, Wv, Wo, which, G, seed, layer, sigma, draws,
+                             Wg=None, E=None) -> np.ndarray:
+    """c[n][t] = -<z~_t - z_t, G_t> for perturbations of `which` (0 q, 1 k, 2 v, 3 the
+    gate's pre-activation, 4 the value embedding); values v = Y Wv^T + s(Y Wg^T) E."""
     Y, Wq, Wk, Wv, Wo, G = (_f32(a) for a in (Y, Wq, Wk, Wv, Wo, G))
+    Wg = None if Wg is None else _f32(Wg)
+    E = None if E is None else _f32(E)
     T, d = Y.shape
     dh = Wq.shape[0]
     off = _i32(seq_offsets)
     draws = _i32(draws)
     c = np.zeros((len(draws), T), np.float64)
-    _check(lib().orc_attention_internal_costs(Y, T, d, off, len(off) - 1, Wq, Wk, Wv, Wo, dh, int(which), G,
+    _check(lib().orc_attention_internal_costs(Y, T, d, off, len(off) - 1, Wq, Wk, Wv, Wo, Wg, E, dh, int(which), G,
                                               seed, layer, float(sigma), draws, len(draws), c),
            "attention_internal_costs")
     return c

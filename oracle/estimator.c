@@ -78,7 +78,7 @@ static int seq_of(const int32_t *off, int n_seq, int t)
 
 int orc_layer_estimate(const float *c_or_r, int is_r, int K, int T, int d_out,
                        const int32_t *seq_offsets, int n_seq, double gamma,
-                       uint32_t seed, uint32_t layer, uint32_t draw_begin,
+                       uint32_t seed, uint32_t layer, uint32_t draw_begin, uint32_t token_begin,
                        int K_total, double sigma,
                        const int32_t *toks, int n_toks,
                        const int32_t *chans, int n_chans, double *g)
@@ -107,7 +107,7 @@ int orc_layer_estimate(const float *c_or_r, int is_r, int K, int T, int d_out,
             }
             for (int m = 0; m < n_chans; ++m) {
                 const uint32_t j = (uint32_t)(chans ? chans[m] : m);
-                const float a = orc_gauss(seed, layer, draw_begin + (uint32_t)k, (uint32_t)t, j, 0);
+                const float a = orc_gauss(seed, layer, draw_begin + (uint32_t)k, token_begin + (uint32_t)t, j, 0);
                 gn[m] += r * (double)a;
             }
         }

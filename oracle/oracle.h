@@ -82,12 +82,14 @@ int orc_reward_scan_brute(const float *c, double *r, int K, int T,
 
 /* ---------------- a5: output-side error estimate [P2, g_t equation] ---------------- */
 
-/* g[n][m] = -(1/(K_total sigma)) sum_{k<K} r[k][toks[n]] a(draw_begin+k, toks[n], chans[m])
+/* g[n][m] = -(1/(K_total sigma)) sum_{k<K} r[k][toks[n]] a(draw_begin+k, token_begin+toks[n], chans[m])
  * where r is c_or_r itself (is_r != 0) or the reward of c_or_r (is_r == 0).
- * c_or_r is [K][T]; chans == NULL means all d_out channels (n_chans = d_out). */
+ * c_or_r is [K][T]; chans == NULL means all d_out channels (n_chans = d_out).
+ * token_begin is the global index of column 0 (a part of a batch split by
+ * sequences draws the noise of its tokens' places in the whole batch). */
 int orc_layer_estimate(const float *c_or_r, int is_r, int K, int T, int d_out,
                        const int32_t *seq_offsets, int n_seq, double gamma,
-                       uint32_t seed, uint32_t layer, uint32_t draw_begin,
+                       uint32_t seed, uint32_t layer, uint32_t draw_begin, uint32_t token_begin,
                        int K_total, double sigma,
                        const int32_t *toks, int n_toks,
                        const int32_t *chans, int n_chans, double *g);
@@ -158,6 +160,7 @@ int orc_toy_suffix_losses(const float *X, const float *W, int T, int d_in, int d
  * channel = projection channel).  Y, G: [T][d]; Wq, Wk, Wv: [dh][d]; Wo: [d][dh]. */
 int orc_attention_internal_costs(const float *Y, int T, int d, const int32_t *offs, int n_seq,
                                  const float *Wq, const float *Wk, const float *Wv, const float *Wo,
+                                 const float *Wg, const float *E,
                                  int dh, int which, const float *G, uint32_t seed, uint32_t layer,
                                  double sigma, const int32_t *draws, int nd, double *c);
 

@@ -18,3 +18,20 @@ def orc():
     import oracle
     oracle.lib()
     return oracle
+
+
+@pytest.fixture(autouse=True)
+def _device_status_after_gpu_tests(request):
+    """After every GPU test, read the status word of each workspace the binding
+    holds: a tcgen05 or fused kernel whose bounded wait ran out records it
+    there, and its output would otherwise look like a result."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    from activation_perturbation_es_b200 import dust
+    if dust._lib is None:
+        return
+    import torch
+    if not torch.cuda.is_available() or not torch.cuda.is_initialized():
+        return
+    assert dust.poll_all() == "ok"

@@ -41,7 +41,7 @@ def test_no_oracle_linkage():
 
 
 def test_status_strings_and_version(L):
-    assert L.dust_abi_version() == 1
+    assert L.dust_abi_version() == 2
     for s, name in dust.STATUS.items():
         assert L.dust_status_string(s).decode() == name
 
@@ -77,16 +77,25 @@ def test_invalid_sizes_rejected_on_host(L):
     assert status(L.dust_layer_estimate(GOOD, 1, 16, 8, GOOD, 1, 0.0, wrap, GOOD, None, 0, None, 0, st)) == 1
     assert status(L.dust_layer_estimate(GOOD, 1, 16, 8, GOOD, 1, 0.0, NZ.c(), None, None, 0, None, 0, st)) == 1
     # head: Vc must divide V and be supported
-    assert status(L.dust_head_step(None, None, 0, GOOD, GOOD, 16, 0, 1000, 300, NZ.c(), None, GOOD, None, None,
-                                   0, GOOD, 1 << 20, st)) == 1
-    assert status(L.dust_head_step(None, None, 0, GOOD, GOOD, 16, 0, 960, 96, NZ.c(), None, GOOD, None, None,
+    assert status(L.dust_head_step(None, None, 0, GOOD, GOOD, 16, 0, 1000, 300, 0, 3, NZ.c(), None, GOOD, None,
+                                   None, 0, GOOD, 1 << 20, st)) == 1
+    assert status(L.dust_head_step(None, None, 0, GOOD, GOOD, 16, 0, 960, 96, 0, 10, NZ.c(), None, GOOD, None, None,
                                    0, GOOD, 1 << 20, st)) == 2
     # Z missing and no X/W to recompute it
-    assert status(L.dust_head_step(None, None, 0, None, GOOD, 16, 8, 512, 128, NZ.c(), None, GOOD, None, None,
+    assert status(L.dust_head_step(None, None, 0, None, GOOD, 16, 8, 512, 128, 0, 4, NZ.c(), None, GOOD, None, None,
                                    0, GOOD, 1 << 20, st)) == 1
+    # chunk ranges outside the V/Vc chunks
+    for cb, cc in ((0, 0), (-1, 2), (3, 2), (4, 1)):
+        assert status(L.dust_head_step(None, None, 0, GOOD, GOOD, 16, 0, 512, 128, cb, cc, NZ.c(), None, GOOD,
+                                       None, None, 0, GOOD, 1 << 20, st)) == 1
+    assert "chunk range" in L.dust_last_error().decode()
+    # token_begin past 2^31
+    far = dust.Noise(0, 0, 0, 4, 4, 0.01, 2**31).c()
+    assert status(L.dust_layer_estimate(GOOD, 1, 16, 8, GOOD, 1, 0.0, far, GOOD, None, 0, None, 0, st)) == 1
     # weight_grad: unknown dtype, zero sizes
-    assert status(L.dust_weight_grad(GOOD, GOOD, 7, 16, 8, 8, GOOD, 0, GOOD, 1 << 20, st)) == 1
-    assert status(L.dust_weight_grad(GOOD, GOOD, 0, 0, 8, 8, GOOD, 0, GOOD, 1 << 20, st)) == 1
+    assert status(L.dust_weight_grad(GOOD, 7, GOOD, 0, 16, 8, 8, GOOD, 0, GOOD, 1 << 20, st)) == 1
+    assert status(L.dust_weight_grad(GOOD, 0, GOOD, 7, 16, 8, 8, GOOD, 0, GOOD, 1 << 20, st)) == 1
+    assert status(L.dust_weight_grad(GOOD, 0, GOOD, 0, 0, 8, 8, GOOD, 0, GOOD, 1 << 20, st)) == 1
     assert "must" in L.dust_last_error().decode()
 
 
@@ -95,7 +104,7 @@ def test_misaligned_pointers_rejected_on_host(L):
     assert status(L.dust_reward_scan(GOOD + 4, GOOD, 4, 16, GOOD, 1, 0.5, st)) == 3
     assert status(L.dust_reward_scan(GOOD, GOOD + 8, 4, 16, GOOD, 1, 0.5, st)) == 3
     assert status(L.dust_layer_estimate(GOOD, 1, 16, 8, GOOD, 1, 0.0, NZ.c(), GOOD + 2, None, 0, None, 0, st)) == 3
-    assert status(L.dust_weight_grad(GOOD, GOOD + 4, 0, 16, 8, 8, GOOD, 0, GOOD, 1 << 20, st)) == 3
+    assert status(L.dust_weight_grad(GOOD, 0, GOOD + 4, 1, 16, 8, 8, GOOD, 0, GOOD, 1 << 20, st)) == 3
     assert "aligned" in L.dust_last_error().decode()
 
 
@@ -104,9 +113,9 @@ def test_workspace_too_small_rejected(L):
     need = L.dust_layer_estimate_workspace(4, 16, 8, 0, 0.9)
     assert need >= 4 * 16 * 4 + 256
     assert status(L.dust_layer_estimate(GOOD, 0, 16, 8, GOOD, 1, 0.9, NZ.c(), GOOD, None, 0, GOOD, need - 1, st)) == 4
-    need = L.dust_head_step_workspace(64, 32, 512, 1, 0, 1)
+    need = L.dust_head_step_workspace(64, 32, 512, 128, 4, 1, 0, 1)
     assert need >= 64 * 512 * 4
-    assert status(L.dust_head_step(GOOD, GOOD, 1, None, GOOD, 64, 32, 512, 128, NZ.c(), None, GOOD, None, GOOD,
+    assert status(L.dust_head_step(GOOD, GOOD, 1, None, GOOD, 64, 32, 512, 128, 0, 4, NZ.c(), None, GOOD, None, GOOD,
                                    0, GOOD, need - 1, st)) == 4
 
 
@@ -116,7 +125,8 @@ def test_workspace_queries_are_consistent(L):
     assert L.dust_layer_estimate_workspace(8, 100, 16, 0, 0.0) == 256
     assert L.dust_layer_estimate_workspace(8, 100, 16, 0, 0.9) >= 256 + 8 * 100 * 4
     # cached Z needs no logits buffer
-    assert L.dust_head_step_workspace(64, 32, 512, 1, 1, 0) < L.dust_head_step_workspace(64, 32, 512, 1, 0, 0)
+    assert L.dust_head_step_workspace(64, 32, 512, 128, 4, 1, 1, 0) < L.dust_head_step_workspace(64, 32, 512, 128, 4,
+                                                                                                  1, 0, 0)
 
 
 def test_fused_estimate_rejected_on_host(L):
@@ -135,6 +145,10 @@ def test_fused_estimate_rejected_on_host(L):
     assert status(f(GOOD, 1, 96, 40, None, 1, 0.0, NZ.c(), GOOD, 128, GOOD, 0, None, GOOD, need - 1, st)) == 4
     need_scan = L.dust_layer_estimate_weight_grad_workspace(4, 96, 128, 40, 0, 0.9)
     assert need_scan >= need + 4 * 96 * 4
+    # one call takes at most 2^20 draws (its bounded waits scale with the draw count)
+    big = dust.Noise(0, 0, 0, (1 << 20) + 1, (1 << 20) + 1, 0.01).c()
+    assert status(f(GOOD, 1, 1, 40, None, 1, 0.0, big, GOOD, 128, GOOD, 0, None, GOOD, 1 << 30, st)) == 2
+    assert "accumulate" in L.dust_last_error().decode()
 
 
 def test_binding_rejects_host_tensors():

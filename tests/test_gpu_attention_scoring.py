@@ -91,3 +91,63 @@ def test_value_estimate_converges_through_uniform_attention():
     g = g.cpu().numpy().astype(np.float64)
     cos = np.sum(g * target) / (np.linalg.norm(g) * np.linalg.norm(target))
     assert cos > 0.98, cos
+
+
+def _gated(p, seed):
+    """Add a gate Wg ~ N(0, 1/d) and value embeddings E ~ N(0, 0.5^2) to a block."""
+    r = np.random.Generator(np.random.PCG64(seed))
+    T, d = p["Y"].shape
+    dh = p["Wq"].shape[0]
+    return dict(p, Wg=(r.standard_normal((dh, d)) * d ** -0.5).astype(np.float32),
+                E=(r.standard_normal((T, dh)) * 0.5).astype(np.float32))
+
+
+@pytest.mark.parametrize("which", [0, 2, 3, 4])
+def test_gate_and_value_embedding_costs_parity(orc, which):
+    """Gated value embeddings on the values: the gate's and the embedding's draws
+    (and q / v draws of the same head) against the oracle."""
+    p = _gated(_block(seed=53), 54)
+    nz = dust.Noise(3, 30 + which, 2, 6, 6, 0.01)
+    c = dust.attention_internal_costs(cu(p["Y"]), cu(p["off"]), cu(p["Wq"]), cu(p["Wk"]), cu(p["Wv"]), cu(p["Wo"]),
+                                      which, cu(p["G"]), nz, Wg=cu(p["Wg"]), E=cu(p["E"])).cpu().numpy()
+    ref = orc.attention_internal_costs(p["Y"], p["off"], p["Wq"], p["Wk"], p["Wv"], p["Wo"], which, p["G"], 3,
+                                       30 + which, 0.01, np.arange(2, 8), Wg=p["Wg"], E=p["E"])
+    assert rel_err(c, ref) < 1e-3
+
+
+def test_gate_and_value_embedding_rejected_without_their_inputs():
+    p = _block(T=64, n_seq=1, d=16, dh=16, seed=55)
+    nz = dust.Noise(0, 1, 0, 2, 2, 0.01)
+    args = [cu(p[k]) for k in ("Y", "off", "Wq", "Wk", "Wv", "Wo")]
+    for which, kw in ((3, {}), (3, {"E": cu(np.zeros((64, 16), np.float32))}), (4, {}), (5, {})):
+        with pytest.raises(dust.DustError) as e:
+            dust.attention_internal_costs(*args, which, cu(p["G"]), nz, **kw)
+        assert e.value.status == 1
+
+
+@pytest.mark.parametrize("which", [3, 4])
+def test_gate_and_value_embedding_estimates_converge(which):
+    """Uniform attention (Wq = Wk = 0), gamma = 1: the estimate approaches the
+    backprop of <z, G> to the perturbed quantity, sum_{s >= t} (G_s Wo)/n_s
+    times s'(g_t) E_t (gate) or s(g_t) (value embedding)."""
+    T, d, dh, K, sigma = 64, 16, 16, 65536, 0.02
+    p = _gated(_block(T=T, n_seq=2, d=d, dh=dh, seed=56), 57)
+    p["Wq"][:] = 0
+    p["Wk"][:] = 0
+    off = p["off"]
+    w = p["G"].astype(np.float64) @ p["Wo"].astype(np.float64)
+    target = np.zeros((T, dh))
+    for q in range(2):
+        for t in range(off[q], off[q + 1]):
+            for s in range(t, off[q + 1]):
+                target[t] += w[s] / (s - off[q] + 1)
+    gp = 1.0 / (1.0 + np.exp(-(p["Y"].astype(np.float64) @ p["Wg"].astype(np.float64).T)))
+    target *= gp * (1 - gp) * p["E"] if which == 3 else gp
+    nz = dust.Noise(6, 40 + which, 0, K, K, sigma)
+    goff = cu(off)
+    c = dust.attention_internal_costs(cu(p["Y"]), goff, cu(p["Wq"]), cu(p["Wk"]), cu(p["Wv"]), cu(p["Wo"]), which,
+                                      cu(p["G"]), nz, Wg=cu(p["Wg"]), E=cu(p["E"]))
+    g, _ = dust.layer_estimate(c, False, goff, 1.0, nz, dh)
+    g = g.cpu().numpy().astype(np.float64)
+    cos = np.sum(g * target) / (np.linalg.norm(g) * np.linalg.norm(target))
+    assert cos > 0.97, cos

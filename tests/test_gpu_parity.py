@@ -203,6 +203,25 @@ def test_weight_grad_bf16_ragged_and_accumulate(orc, T, d_in, d_out):
     assert rel_err(host(G), ref) < 1e-5
 
 
+@pytest.mark.parametrize("g_bf16", [False, True])
+@pytest.mark.parametrize("T,d_in,d_out", [(1000, 72, 40), (4096, 256, 130)])
+def test_weight_grad_mixed_dtypes(orc, g_bf16, T, d_in, d_out):
+    """fp32 g with bf16 X and bf16 g with fp32 X (the reduction's fp32 g against
+    a bf16 layer input, or its bf16 copy against an fp32 input): the bf16
+    operand is widened exactly, so the bar is fp32 accumulation's."""
+    g = I.normal((T, d_out), 1.0, seed=T + 11)
+    X = I.normal((T, d_in), 1.0, seed=T + 12)
+    if g_bf16:
+        g = I.bf16_round(g)
+    else:
+        X = I.bf16_round(X)
+    G0 = I.normal((d_out, d_in), 1.0, seed=T + 13)
+    G = cu(G0)
+    dust.weight_grad(cu(g, torch.bfloat16 if g_bf16 else torch.float32),
+                     cu(X, torch.float32 if g_bf16 else torch.bfloat16), G_W=G, accumulate=True)
+    assert rel_err(host(G), orc.weight_grad(g, X) + G0.astype(np.float64)) < 1e-5
+
+
 @pytest.mark.parametrize("T,d_in,V", [(1000, 64, 520), (256, 1024, 4096)])
 def test_logits_bf16_tensor_cores(orc, T, d_in, V):
     X = I.bf16_round(I.normal((T, d_in), 1.0, seed=T))
@@ -304,11 +323,17 @@ def test_head_pages_sampled(orc, K):
     c_ref, g_ref = orc.head_step(Zs, h["y"][toks], toks, w.Vc, nz.seed, nz.layer, 0, K, K, w.sigma)
     assert rel_err(host(out["g_hat"])[toks], g_ref) < FP32_TOL
     assert rel_err(host(out["c"])[:, :, toks], c_ref) < FP32_TOL
-    # G_W is the weight GEMM of the kernel's bf16 g (the GEMM at this shape is
-    # pinned against the oracle on seeded inputs in test_weight_grad_bf16; a
-    # vocabulary column of g over all 16384 tokens is beyond the oracle)
-    G2 = dust.weight_grad(out["g_hat_bf16"], X)
-    assert rel_err(host(out["G_W"]), host(G2).astype(np.float64)) < 1e-6
+    # G_W rows against the oracle's chain: its g over all 16384 tokens (the
+    # logits are the float64 product X W^T, rounded to binary32 as the oracle's
+    # logits are), held in binary32 and rounded to bf16 as the kernels hold it
+    X64, W64 = h["X"].astype(np.float64), h["W"].astype(np.float64)
+    Z_all = (X64 @ W64.T).astype(np.float32)
+    _, g_all = orc.head_step(Z_all, h["y"], np.arange(w.T), w.Vc, nz.seed, nz.layer, 0, K, K, w.sigma,
+                             want_c=False)
+    rows = np.sort(np.random.Generator(np.random.PCG64(8)).choice(w.V, 8, replace=False))
+    g_rows = torch.from_numpy(np.ascontiguousarray(g_all[:, rows]).astype(np.float32)).to(torch.bfloat16)
+    G_ref = orc.weight_grad(g_rows.float().numpy(), h["X"], rows=np.arange(len(rows)))
+    assert rel_err(host(out["G_W"])[rows], G_ref) < 1e-3
 
 
 # ------------------------------------------------------------------ hidden layer, config-sized

@@ -73,3 +73,36 @@ def test_sigma_sweep(orc):
     assert best in (1e-3, 1e-2, 1e-1)
     assert coss[-1] < max(coss[:-1])            # far outside the first-order regime the cosine drops
     assert abs(coss[0] - coss[1]) < 0.05        # inside it the cosine barely depends on sigma
+
+
+def test_hidden_sweep_picks_gamma_one_against_backprop(orc):
+    """A hidden layer of the toy causal suffix (2 sequences x 16 tokens): the
+    caller scores its perturbed forward (the library's toy suffix) and supplies
+    -grad_W sum l from float64 autograd; against the full backprop gradient the
+    discount that keeps every later token's loss, gamma = 1, wins, and each
+    cosine matches the oracle chain's on the same costs."""
+    import suffix_autograd as SA
+    p = SA.tiny_problem()
+    G_ref = -SA.backprop_gradient(p)
+    cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    Y = dust.logits(cu(p["X"]), cu(p["W"]))
+    off = cu(p["off"])
+
+    def costs(nz):
+        return dust.toy_suffix_losses(Y, off, cu(p["Wq"]), cu(p["Wk"]), cu(p["Wv"]), cu(p["Wo"]), cu(p["Wout"]),
+                                      cu(p["y"]), nz)[1]
+
+    K, d = 8192, p["W"].shape[0]
+    sigmas, gammas = [1e-3, 1e-2], [0.0, 0.5, 0.9, 1.0]
+    _, _, coss, best = tuner.hidden_sweep(costs, cu(p["X"]), off, d, cu(G_ref.astype(np.float32)), K, sigmas,
+                                          gammas, seed=0, layer=5)
+    assert best[1] == 1.0, coss
+    assert np.all(np.diff(coss, axis=1) > 0), coss           # more of the future helps, for either sigma
+    assert coss[1, -1] > 0.99, coss
+    # the sweep's cosine at (1e-2, 0.9) against the oracle's chain on the same costs
+    c = costs(dust.Noise(0, 5, 0, K, K, 1e-2)).cpu().numpy()
+    T = p["X"].shape[0]
+    g = orc.layer_estimate(c, False, d, p["off"], 0.9, 0, 5, 0, K, 1e-2, np.arange(T))
+    G = orc.weight_grad(g.astype(np.float32), p["X"])
+    ref = np.sum(G * G_ref) / (np.linalg.norm(G) * np.linalg.norm(G_ref))
+    assert abs(coss[1, 2] - ref) < 2e-3, (coss[1, 2], ref)

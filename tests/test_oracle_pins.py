@@ -69,6 +69,11 @@ def test_estimate_single_draw_closed_form(orc):
     g = orc.layer_estimate(np.array([[r]], np.float32), True, 8, [0, 1], 0.0, 5, 3, 11, 1, sigma, [0])
     a = np.array([orc.gauss(5, 3, 11, 0, j) for j in range(8)], np.float64)
     np.testing.assert_allclose(g[0], -(float(np.float32(r)) / sigma) * a, rtol=1e-15)
+    # the same token placed at global index 70000 of a sharded batch draws that token's noise
+    g = orc.layer_estimate(np.array([[r]], np.float32), True, 8, [0, 1], 0.0, 5, 3, 11, 1, sigma, [0],
+                           token_begin=70000)
+    a = np.array([orc.gauss(5, 3, 11, 70000, j) for j in range(8)], np.float64)
+    np.testing.assert_allclose(g[0], -(float(np.float32(r)) / sigma) * a, rtol=1e-15)
 
 
 def test_estimate_reward_path_and_draw_split(orc):
@@ -392,6 +397,89 @@ def test_attention_value_estimate_converges_to_backprop_through_uniform_attentio
     Kmax = 8192
     c = orc.attention_internal_costs(p["Y"], off, p["Wq"], p["Wk"], p["Wv"], p["Wo"], 2, p["G"], 1, 7, sigma,
                                      np.arange(Kmax)).astype(np.float32)
+    errs = []
+    Ks = [128, 512, 2048, 8192]
+    for K in Ks:
+        g = orc.layer_estimate(c[:K], False, dh, off, 1.0, 1, 7, 0, K, sigma, np.arange(T))
+        errs.append(np.linalg.norm(g - target) / np.linalg.norm(target))
+    slope = np.polyfit(np.log(Ks), np.log(errs), 1)[0]
+    assert -0.6 <= slope <= -0.4, (slope, errs)
+    assert errs[-1] < 0.2, errs
+
+
+def _gated_values(seed=43, T=14, d=8, dh=4):
+    p = _attn_small(seed=seed, T=T, d=d, dh=dh)
+    r = np.random.Generator(np.random.PCG64(seed + 100))
+    p["Wg"] = (r.standard_normal((dh, d)) * 0.5).astype(np.float32)
+    p["E"] = (r.standard_normal((T, dh)) * 0.7).astype(np.float32)
+    return p
+
+
+def _costs(orc, p, which, sigma, draws, seed=0, layer=5, off=None):
+    return orc.attention_internal_costs(p["Y"], p["off"] if off is None else off, p["Wq"], p["Wk"], p["Wv"], p["Wo"],
+                                        which, p["G"], seed, layer, sigma, draws, Wg=p.get("Wg"), E=p.get("E"))
+
+
+def test_gate_and_value_embedding_special_cases(orc):
+    """The gate matters only through the value embedding (E = 0: every gate cost
+    is 0); with Wg = 0 the gate is s(0) = 1/2 everywhere, so a value-embedding
+    draw moves v by half of what the same draw does to the value projection,
+    and since the attention output is linear in v its costs are half the
+    value-projection costs (under any q, k)."""
+    p = _gated_values()
+    p0 = dict(p, E=np.zeros_like(p["E"]))
+    assert np.all(_costs(orc, p0, 3, 0.1, [0, 4]) == 0.0)
+    ph = dict(p, Wg=np.zeros_like(p["Wg"]))
+    np.testing.assert_allclose(_costs(orc, ph, 4, 0.1, [1, 2]), 0.5 * _costs(orc, ph, 2, 0.1, [1, 2]), rtol=1e-10,
+                               atol=1e-15)
+    # the clean values carry the gated embedding: q draws see it (their costs change with E)
+    assert not np.allclose(_costs(orc, p, 0, 0.1, [3]), _costs(orc, p0, 0, 0.1, [3]))
+
+
+@pytest.mark.parametrize("which", [3, 4])
+def test_gate_and_value_embedding_uniform_attention_closed_form(orc, which):
+    """Wq = Wk = 0: the output change is the causal running mean of the values'
+    change, (s(g + sigma a) - s(g)) e for the gate and s(g) sigma a for the value
+    embedding (numpy, scipy's logistic function)."""
+    p = _gated_values()
+    p["Wq"] = np.zeros_like(p["Wq"])
+    p["Wk"] = np.zeros_like(p["Wk"])
+    sigma, T, dh = 0.3, p["Y"].shape[0], p["Wq"].shape[0]
+    c = _costs(orc, p, which, sigma, [5])
+    a = orc.noise_block(0, 5, 5, 1, np.arange(T), 0, dh)[0].astype(np.float64)
+    g = p["Y"].astype(np.float64) @ p["Wg"].astype(np.float64).T
+    dv = (sp.expit(g + sigma * a) - sp.expit(g)) * p["E"] if which == 3 else sp.expit(g) * sigma * a
+    dz = np.zeros((T, p["Y"].shape[1]))
+    off = p["off"]
+    for q in range(len(off) - 1):
+        seg = dv[off[q]:off[q + 1]]
+        if len(seg):
+            m = np.cumsum(seg, axis=0) / np.arange(1, len(seg) + 1)[:, None]
+            dz[off[q]:off[q + 1]] = m @ p["Wo"].astype(np.float64).T
+    np.testing.assert_allclose(c[0], -np.sum(dz * p["G"], axis=1), rtol=1e-10, atol=1e-14)
+
+
+@pytest.mark.parametrize("which", [3, 4])
+def test_gate_and_value_embedding_estimates_converge_to_backprop(orc, which):
+    """Uniform attention, gamma = 1: the estimate's expectation is the backprop of
+    <z, G> to the perturbed quantity, the value path's sum_{s >= t} (G_s Wo)/n_s
+    times dv/dx: s'(g) e for the gate, s(g) for the value embedding (first
+    order in sigma).  The error falls like K^-1/2."""
+    p = _gated_values(seed=44, T=10, d=6, dh=8)
+    p["Wq"] = np.zeros_like(p["Wq"])
+    p["Wk"] = np.zeros_like(p["Wk"])
+    off = np.array([0, 4, 10], np.int32)
+    T, dh, sigma = 10, 8, 0.02
+    w = p["G"].astype(np.float64) @ p["Wo"].astype(np.float64)
+    target = np.zeros((T, dh))
+    for q in range(2):
+        for t in range(off[q], off[q + 1]):
+            for s in range(t, off[q + 1]):
+                target[t] += w[s] / (s - off[q] + 1)
+    gp = sp.expit(p["Y"].astype(np.float64) @ p["Wg"].astype(np.float64).T)
+    target *= gp * (1 - gp) * p["E"] if which == 3 else gp
+    Kmax = 8192
+    c = _costs(orc, p, which, sigma, np.arange(Kmax), seed=1, layer=7, off=off).astype(np.float32)
     errs = []
     Ks = [128, 512, 2048, 8192]
     for K in Ks:

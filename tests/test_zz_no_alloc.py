@@ -31,22 +31,30 @@ def rel_err(a, b):
     return float(np.max(np.abs(a - b)) / np.max(np.abs(b)))
 
 
-def test_noalloc_matches_workspace_entry_point_twice():
-    cases = [  # two calls in a row with different shapes, costs and discounts
+def test_noalloc_matches_workspace_entry_point_twice(orc):
+    """Two calls in a row with different shapes, costs and discounts: the same
+    bits as dust_layer_estimate (the same kernels on the same rewards; the
+    third case takes the chunked scan in both), and the oracle's values."""
+    cases = [
         (I.offsets_from_lengths([700, 0, 301, 23]), 48, 0.95, 1000, 3),
         (I.uniform_offsets(4, 256), 130, 0.5, 32, 7),
+        (I.uniform_offsets(1, 5000), 20, 0.9, 16, 9),        # few long sequences: chunked scan
     ]
     for off, d_out, gamma, K, seed in cases:
         T = int(off[-1])
-        c = torch.from_numpy(I.normal((K, T), 0.01, seed=seed)).cuda()
+        c_np = I.normal((K, T), 0.01, seed=seed)
+        c = torch.from_numpy(c_np).cuda()
         goff = torch.from_numpy(off).cuda()
         nz = dust.Noise(seed, 5, 0, K, K, 0.01)
         ref, ref16 = dust.layer_estimate(c, False, goff, gamma, nz, d_out, g_hat_bf16=True)
         g16 = torch.empty(T, d_out, dtype=torch.bfloat16, device="cuda")
         got, got16 = dust.layer_estimate_noalloc(c, goff, gamma, nz, d_out, g_hat_bf16=g16)
         torch.cuda.synchronize()
-        assert rel_err(got, ref) < FP32_TOL
-        assert rel_err(got16, ref16) < FP32_TOL
+        assert torch.equal(got, ref)
+        assert torch.equal(got16, ref16)
+        toks = np.array([0, T // 2, T - 1])
+        g_orc = orc.layer_estimate(c_np, False, d_out, off, gamma, seed, 5, 0, K, 0.01, toks)
+        assert rel_err(got[toks], torch.from_numpy(g_orc)) < FP32_TOL
 
 
 def test_noalloc_rejects_sizes_beyond_the_scratch():
