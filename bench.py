@@ -73,6 +73,17 @@ SLOTS_A5 = (111 + 4) / 4               # 28.75 per Gaussian
 SLOTS_HEAD = (111 + 15) / 4            # 31.5 per perturbed logit
 LANES_PER_SM = 128                     # 4 schedulers x 32 lanes
 
+# The same work on the datapath that binds both ALU kernels, the FMA-heavy one:
+# a packed fp32 instruction holds it (and FMA-lite) for 2 cycles, a 32x32->64
+# product holds it for 4 (ncu's active-cycle and instruction counters fit these
+# costs).  Per Philox call, with every product the specification needs, less
+# those that no draw changes: 18 products in the reduction (round 1's quad
+# product is draw-invariant, its draw product steps by an add), 18 1/8 in the
+# head (the draw product is shared by a lane's 8 quads); packed operations:
+# 34 in the generator, 3 in the reduction's consumer and 14 in the head's.
+HEAVY_A5 = (18 * 4 + (34 + 3) * 2) / 4          # 36.5 heavy cycles per Gaussian
+HEAVY_HEAD = (18.125 * 4 + (34 + 14) * 2) / 4   # 42.125 per perturbed logit
+
 
 def parse_args():
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
@@ -443,7 +454,8 @@ def main():
                                      "accumulation in TMEM (tcgen05)"},
             "roofline": {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
             | {"kernel": dominant["name"], "clock_mhz_for_peak": dominant.get("clock_mhz_for_peak"),
-               "peak_source": dominant.get("peak_source")},
+               "peak_source": dominant.get("peak_source"),
+               "fma_heavy_pipe": dominant.get("fma_heavy_pipe")},
             "kernels": kernels,
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -576,6 +588,14 @@ def kernel_report(step, stages, peaks, clocks):
                     "peak_source": "148 SMs x 4 schedulers x 32 lanes x max SM clock (one issue slot per lane "
                                    "per clock); work = the specification's operations in their cheapest sm_100 "
                                    "instruction forms"}
+            # the binding datapath's view of the same kernel: the specification's FMA-heavy cycles
+            # against one cycle per lane per scheduler; the issue-slot fraction above cannot exceed
+            # slots_per_element / heavy_cycles_per_element on sm_100
+            heavy_el = HEAVY_HEAD if layer == "head" else HEAVY_A5
+            rec["fma_heavy_pipe"] = {
+                "cycles_per_element": heavy_el,
+                "frac": float(K) * T * d_out * heavy_el / (ms / 1e3) / 1e12 / alu_peak,
+                "issue_slot_frac_cap": slots_el / heavy_el}
         out.append(rec)
     return out
 
