@@ -7,7 +7,7 @@ import torch
 
 
 def weight_rows(orc, c_or_r, is_r, d_out, offsets, gamma, seed, layer, draw_begin, K_total, sigma, X, rows,
-                bf16=True):
+                bf16=True, token_begin=0):
     """Rows `rows` of G_W = sum_t g_t x_t^T, with g_t[rows] from the oracle's
     estimate over every token.  g is taken to binary32 and, for the bf16
     weight GEMM, rounded to bf16 (nearest, ties to even): the precisions in
@@ -20,7 +20,7 @@ def weight_rows(orc, c_or_r, is_r, d_out, offsets, gamma, seed, layer, draw_begi
         # the kernels hold r, instead of one recurrence per token
         c_or_r = orc.reward_scan(c_or_r, offsets, gamma).astype(np.float32)
     g = orc.layer_estimate(c_or_r, True, d_out, offsets, gamma, seed, layer, draw_begin, K_total, sigma,
-                           np.arange(T), chans=rows).astype(np.float32)
+                           np.arange(T), chans=rows, token_begin=token_begin).astype(np.float32)
     if bf16:
         # round to nearest bf16, ties to even (torch's CPU conversion)
         g = torch.from_numpy(g).to(torch.bfloat16).float().numpy()

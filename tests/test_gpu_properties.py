@@ -1,7 +1,8 @@
 """GPU parity on random small shapes (hypothesis, derandomized so every run
 draws the same examples): ragged and empty sequences, odd token counts,
 channel counts not divisible by 4, draw ranges split over calls, gamma's
-special values, vocabulary chunk counts, and the fused reduction + weight
+special values, vocabulary chunk counts and chunk ranges, tokens placed at
+random global offsets (token_begin), and the fused reduction + weight
 estimate.  Every expected value comes from the oracle on the same seeded
 inputs."""
 import numpy as np
@@ -43,52 +44,57 @@ def cu(a, dtype=None):
 
 @settings(**SETTINGS)
 @given(lengths=lengths_st, d_out=st.integers(1, 70), K=st.integers(1, 9), split=st.integers(1, 8),
-       gamma=gamma_st, seed=st.integers(0, 10_000))
-def test_estimate_random_shapes(orc, lengths, d_out, K, split, gamma, seed):
+       gamma=gamma_st, seed=st.integers(0, 10_000), tb=st.integers(0, 2**31 - 1000))
+def test_estimate_random_shapes(orc, lengths, d_out, K, split, gamma, seed, tb):
     """Scan + reduction against the oracle, with the draws split over two
-    calls (accumulate = 1) at a random point."""
+    calls (accumulate = 1) at a random point and the tokens at global offset tb."""
     off = I.offsets_from_lengths(lengths)
     T = int(off[-1])
     c = I.normal((K, T), 0.02, seed=seed)
     a = min(split, K)
-    nz_all = dust.Noise(seed % 7, 3, 5, K, K, 0.01)
+    nz_all = dust.Noise(seed % 7, 3, 5, K, K, 0.01, tb)
     goff = cu(off)
-    g, _ = dust.layer_estimate(cu(c[:a]), False, goff, gamma, dust.Noise(seed % 7, 3, 5, a, K, 0.01), d_out)
+    g, _ = dust.layer_estimate(cu(c[:a]), False, goff, gamma, dust.Noise(seed % 7, 3, 5, a, K, 0.01, tb), d_out)
     if a < K:
-        dust.layer_estimate(cu(c[a:]), False, goff, gamma, dust.Noise(seed % 7, 3, 5 + a, K - a, K, 0.01), d_out,
-                            g_hat=g, accumulate=True)
-    ref = orc.layer_estimate(c, False, d_out, off, gamma, nz_all.seed, 3, 5, K, 0.01, np.arange(T))
+        dust.layer_estimate(cu(c[a:]), False, goff, gamma, dust.Noise(seed % 7, 3, 5 + a, K - a, K, 0.01, tb),
+                            d_out, g_hat=g, accumulate=True)
+    ref = orc.layer_estimate(c, False, d_out, off, gamma, nz_all.seed, 3, 5, K, 0.01, np.arange(T), token_begin=tb)
     assert rel_err(g.cpu().numpy(), ref) < FP32_TOL
 
 
 @settings(**dict(SETTINGS, max_examples=40))
 @given(T=st.integers(1, 40), n_chunks=st.integers(1, 4), Vc=st.sampled_from([128, 256, 384, 1024]),
-       K=st.integers(1, 6), sigma=st.sampled_from([0.005, 0.02, 0.05]), seed=st.integers(0, 10_000))
-def test_head_random_shapes(orc, T, n_chunks, Vc, K, sigma, seed):
-    """Head step (cached logits) against the oracle: c per chunk and g."""
+       K=st.integers(1, 6), sigma=st.sampled_from([0.005, 0.02, 0.05]), seed=st.integers(0, 10_000),
+       first=st.integers(0, 3), tb=st.integers(0, 2**31 - 1000))
+def test_head_random_shapes(orc, T, n_chunks, Vc, K, sigma, seed, first, tb):
+    """Head step (cached logits) over a random range of its chunks, with the
+    tokens at global offset tb, against the oracle: c per chunk and g."""
     V = n_chunks * Vc
+    cb = first % n_chunks
+    cc = n_chunks - cb
     Z = I.normal((T, V), 1.5, seed=seed)
     y = I.targets(T, V, seed=seed + 1)
-    nz = dust.Noise(seed % 5, 9, 2, K, K, sigma)
-    out = dust.head_step(cu(y), Vc, nz, Z=cu(Z), want_c=True)
-    c_ref, g_ref = orc.head_step(Z, y, np.arange(T), Vc, nz.seed, nz.layer, 2, K, K, sigma)
-    assert rel_err(out["g_hat"].cpu().numpy(), g_ref) < FP32_TOL
-    assert rel_err(out["c"].cpu().numpy(), c_ref) < FP32_TOL
+    nz = dust.Noise(seed % 5, 9, 2, K, K, sigma, tb)
+    out = dust.head_step(cu(y), Vc, nz, Z=cu(Z), want_c=True, chunk_begin=cb, chunk_count=cc)
+    c_ref, g_ref = orc.head_step(Z, y, tb + np.arange(T), Vc, nz.seed, nz.layer, 2, K, K, sigma)
+    assert rel_err(out["g_hat"].cpu().numpy(), g_ref[:, cb * Vc:]) < FP32_TOL
+    assert rel_err(out["c"].cpu().numpy(), c_ref[cb:]) < FP32_TOL
 
 
 @settings(**dict(SETTINGS, max_examples=30))
 @given(lengths=lengths_st, d_out=st.integers(1, 300), d_in=st.sampled_from([64, 128, 192, 256, 320, 384, 448, 512]),
-       K=st.integers(1, 7), gamma=gamma_st, seed=st.integers(0, 10_000))
-def test_fused_random_shapes(orc, lengths, d_out, d_in, K, gamma, seed):
-    """Fused reduction + weight estimate against the oracle's chain."""
+       K=st.integers(1, 7), gamma=gamma_st, seed=st.integers(0, 10_000), tb=st.integers(0, 2**31 - 1000))
+def test_fused_random_shapes(orc, lengths, d_out, d_in, K, gamma, seed, tb):
+    """Fused reduction + weight estimate against the oracle's chain (tokens at global offset tb)."""
     off = I.offsets_from_lengths(lengths)
     T = int(off[-1])
     c = I.normal((K, T), 0.02, seed=seed)
     X = I.bf16_round(I.normal((T, d_in), 1.0, seed=seed + 1))
-    nz = dust.Noise(seed % 3, 4, 0, K, K, 0.01)
+    nz = dust.Noise(seed % 3, 4, 0, K, K, 0.01, tb)
     G, g = dust.layer_estimate_weight_grad(cu(c), False, cu(off), gamma, nz, cu(X, torch.bfloat16), d_out,
                                            g_hat=True)
-    g_ref = orc.layer_estimate(c, False, d_out, off, gamma, nz.seed, 4, 0, K, 0.01, np.arange(T))
+    g_ref = orc.layer_estimate(c, False, d_out, off, gamma, nz.seed, 4, 0, K, 0.01, np.arange(T), token_begin=tb)
     assert rel_err(g.cpu().numpy(), g_ref) < FP32_TOL
-    G_ref = oracle_chains.weight_rows(orc, c, False, d_out, off, gamma, nz.seed, 4, 0, K, 0.01, X, np.arange(d_out))
+    G_ref = oracle_chains.weight_rows(orc, c, False, d_out, off, gamma, nz.seed, 4, 0, K, 0.01, X, np.arange(d_out),
+                                      token_begin=tb)
     assert rel_err(G.cpu().numpy(), G_ref) < FP32_TOL
