@@ -36,53 +36,59 @@ def _nullable(kind):
 def lib():
     global _lib
     if _lib is None:
-        L = C.CDLL(build())
-        u32, i32, dbl, flt = C.c_uint32, C.c_int, C.c_double, C.c_float
-        L.orc_philox4x32_10.argtypes = [_u32p, _u32p, _u32p]
-        L.orc_ln.argtypes = [flt]
-        L.orc_ln.restype = flt
-        L.orc_sincos_quarter.argtypes = [flt, C.POINTER(flt), C.POINTER(flt)]
-        L.orc_box_muller.argtypes = [u32, u32, C.POINTER(flt), C.POINTER(flt)]
-        L.orc_philox_batch.argtypes = [_u32p, _u32p, i32, _u32p]
-        L.orc_ln_batch.argtypes = [_f32p, i32, _f32p]
-        L.orc_sincos_batch.argtypes = [_f32p, i32, _f32p, _f32p]
-        L.orc_box_muller_batch.argtypes = [_u32p, _u32p, i32, _f32p, _f32p]
-        L.orc_gauss.argtypes = [u32] * 6
-        L.orc_gauss.restype = flt
-        L.orc_noise_block.argtypes = [u32, u32, u32, u32, i32, _i32p, i32, u32, i32, _f32p]
-        L.orc_reward_scan.argtypes = [_f32p, _f64p, i32, i32, _i32p, i32, dbl]
-        L.orc_reward_scan.restype = i32
-        L.orc_reward_scan_brute.argtypes = [_f32p, _f64p, i32, i32, _i32p, i32, dbl]
-        L.orc_reward_scan_brute.restype = i32
-        L.orc_layer_estimate.argtypes = [_f32p, i32, i32, i32, i32, _i32p, i32, dbl,
-                                         u32, u32, u32, u32, i32, dbl, _i32p, i32,
-                                         _nullable(_i32p), i32, _f64p]
-        L.orc_layer_estimate.restype = i32
-        L.orc_weight_grad.argtypes = [_f32p, _f32p, i32, i32, i32, _i32p, i32, _f64p]
-        L.orc_weight_grad.restype = i32
-        L.orc_logits.argtypes = [_f32p, _f32p, i32, i32, i32, _i32p, i32, _f64p]
-        L.orc_logits.restype = i32
-        L.orc_head_clean.argtypes = [_f32p, _i32p, i32, i32, _f64p, _f64p]
-        L.orc_head_clean.restype = i32
-        L.orc_head_step.argtypes = [_f32p, _i32p, _i32p, i32, i32, i32, u32, u32, u32, i32,
-                                    i32, dbl, _nullable(_f64p), _f64p]
-        L.orc_head_step.restype = i32
-        L.orc_head_bp_grad.argtypes = [_f32p, _i32p, _f32p, i32, i32, i32, _i32p, i32, _f64p]
-        L.orc_head_bp_grad.restype = i32
-        L.orc_cosine.argtypes = [_f32p, _f32p, C.c_longlong]
-        L.orc_cosine.restype = dbl
-        L.orc_synth_costs.argtypes = [_f32p, i32, i32, u32, u32, dbl, dbl, _i32p, _i32p, i32, _f64p]
-        L.orc_synth_costs.restype = i32
-        L.orc_toy_suffix_losses.argtypes = [_f32p, _f32p, i32, i32, i32, _i32p, i32,
-                                            _f32p, _f32p, _f32p, _f32p, i32, _f32p, i32,
-                                            _i32p, u32, u32, dbl, i32, _i32p, i32, _f64p]
-        L.orc_toy_suffix_losses.restype = i32
-        L.orc_attention_internal_costs.argtypes = [_f32p, i32, i32, _i32p, i32, _f32p, _f32p, _f32p, _f32p,
-                                                   _nullable(_f32p), _nullable(_f32p), i32, i32,
-                                                   _f32p, u32, u32, dbl, _i32p, i32, _f64p]
-        L.orc_attention_internal_costs.restype = i32
-        _lib = L
+        _lib = load(build())
     return _lib
+
+
+def load(path: str) -> C.CDLL:
+    """Load an oracle library built from these sources (the tests also load
+    deliberately broken builds, to show that the pins catch them)."""
+    L = C.CDLL(path)
+    u32, i32, dbl, flt = C.c_uint32, C.c_int, C.c_double, C.c_float
+    L.orc_philox4x32_10.argtypes = [_u32p, _u32p, _u32p]
+    L.orc_ln.argtypes = [flt]
+    L.orc_ln.restype = flt
+    L.orc_sincos_quarter.argtypes = [flt, C.POINTER(flt), C.POINTER(flt)]
+    L.orc_box_muller.argtypes = [u32, u32, C.POINTER(flt), C.POINTER(flt)]
+    L.orc_philox_batch.argtypes = [_u32p, _u32p, i32, _u32p]
+    L.orc_ln_batch.argtypes = [_f32p, i32, _f32p]
+    L.orc_sincos_batch.argtypes = [_f32p, i32, _f32p, _f32p]
+    L.orc_box_muller_batch.argtypes = [_u32p, _u32p, i32, _f32p, _f32p]
+    L.orc_gauss.argtypes = [u32] * 6
+    L.orc_gauss.restype = flt
+    L.orc_noise_block.argtypes = [u32, u32, u32, u32, i32, _i32p, i32, u32, i32, _f32p]
+    L.orc_reward_scan.argtypes = [_f32p, _f64p, i32, i32, _i32p, i32, dbl]
+    L.orc_reward_scan.restype = i32
+    L.orc_reward_scan_brute.argtypes = [_f32p, _f64p, i32, i32, _i32p, i32, dbl]
+    L.orc_reward_scan_brute.restype = i32
+    L.orc_layer_estimate.argtypes = [_f32p, i32, i32, i32, i32, _i32p, i32, dbl,
+                                     u32, u32, u32, u32, i32, dbl, _i32p, i32,
+                                     _nullable(_i32p), i32, _f64p]
+    L.orc_layer_estimate.restype = i32
+    L.orc_weight_grad.argtypes = [_f32p, _f32p, i32, i32, i32, _i32p, i32, _f64p]
+    L.orc_weight_grad.restype = i32
+    L.orc_logits.argtypes = [_f32p, _f32p, i32, i32, i32, _i32p, i32, _f64p]
+    L.orc_logits.restype = i32
+    L.orc_head_clean.argtypes = [_f32p, _i32p, i32, i32, _f64p, _f64p]
+    L.orc_head_clean.restype = i32
+    L.orc_head_step.argtypes = [_f32p, _i32p, _i32p, i32, i32, i32, u32, u32, u32, i32,
+                                i32, dbl, _nullable(_f64p), _f64p]
+    L.orc_head_step.restype = i32
+    L.orc_head_bp_grad.argtypes = [_f32p, _i32p, _f32p, i32, i32, i32, _i32p, i32, _f64p]
+    L.orc_head_bp_grad.restype = i32
+    L.orc_cosine.argtypes = [_f32p, _f32p, C.c_longlong]
+    L.orc_cosine.restype = dbl
+    L.orc_synth_costs.argtypes = [_f32p, i32, i32, u32, u32, dbl, dbl, _i32p, _i32p, i32, _f64p]
+    L.orc_synth_costs.restype = i32
+    L.orc_toy_suffix_losses.argtypes = [_f32p, _f32p, i32, i32, i32, _i32p, i32,
+                                        _f32p, _f32p, _f32p, _f32p, i32, _f32p, i32,
+                                        _i32p, u32, u32, dbl, i32, _i32p, i32, _f64p]
+    L.orc_toy_suffix_losses.restype = i32
+    L.orc_attention_internal_costs.argtypes = [_f32p, i32, i32, _i32p, i32, _f32p, _f32p, _f32p, _f32p,
+                                               _nullable(_f32p), _nullable(_f32p), i32, i32,
+                                               _f32p, u32, u32, dbl, _i32p, i32, _f64p]
+    L.orc_attention_internal_costs.restype = i32
+    return L
 
 
 def _f32(a):

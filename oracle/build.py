@@ -24,13 +24,19 @@ def _stale() -> bool:
     return any(os.path.getmtime(os.path.join(HERE, s)) > t for s in deps)
 
 
+def compile_sources(src_dir: str, out: str) -> str:
+    """Compile the oracle's sources found in src_dir into the shared library out."""
+    cmd = ["gcc", "-O2", "-std=gnu11", "-fPIC", "-shared", "-fopenmp",
+           "-ffp-contract=off", "-fno-fast-math", "-Wall", "-Wextra",
+           "-o", out + ".tmp"] + [os.path.join(src_dir, s) for s in SOURCES] + ["-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(out + ".tmp", out)
+    return out
+
+
 def build(force: bool = False) -> str:
     if force or _stale():
-        cmd = ["gcc", "-O2", "-std=gnu11", "-fPIC", "-shared", "-fopenmp",
-               "-ffp-contract=off", "-fno-fast-math", "-Wall", "-Wextra",
-               "-o", LIB + ".tmp"] + [os.path.join(HERE, s) for s in SOURCES] + ["-lm"]
-        subprocess.run(cmd, check=True)
-        os.replace(LIB + ".tmp", LIB)
+        compile_sources(HERE, LIB)
     return LIB
 
 
