@@ -596,6 +596,10 @@ def kernel_report(step, stages, peaks, clocks):
                 "cycles_per_element": heavy_el,
                 "frac": float(K) * T * d_out * heavy_el / (ms / 1e3) / 1e12 / alu_peak,
                 "issue_slot_frac_cap": slots_el / heavy_el}
+            # and HBM's: the bytes the kernel must move over its time, against the copy bandwidth
+            # (small by construction: the noise is regenerated, never read)
+            gbs = alg_bytes / (ms / 1e3) / 1e9
+            rec["hbm"] = {"achieved_gbs": gbs, "frac": gbs / peaks["hbm_gbs"]}
         out.append(rec)
     return out
 
