@@ -47,8 +47,13 @@ def test_draw_split_of_the_hidden_sweep():
     parts = [_run(w, K, r, 2, "draws") for r in range(2)]
     assert [p.draws for p in parts] == [32, 32]
     for i, L in enumerate(whole.hidden):
+        # the fp32 error estimate is linear in the draws: the ranks' parts add up to the whole
+        g = sum(p.hidden[i]["g"].double() for p in parts).cpu().numpy()
+        assert rel_err(g, L["g"].cpu().numpy()) < 1e-5, L["hl"].name
+        # each rank rounds its own part of g to bf16 for the tensor-core GEMM, so the summed weight
+        # estimates differ from the whole's by bf16 rounding (2^-8 relative), the bf16 GEMM path's bar
         G = sum(p.hidden[i]["G"].double() for p in parts).cpu().numpy()
-        assert rel_err(G, L["G"].cpu().numpy()) < 1e-4, L["hl"].name   # bf16 g, two fp32 sums
+        assert rel_err(G, L["G"].cpu().numpy()) < 2e-2, L["hl"].name
 
 
 def test_vocabulary_split_of_the_head():
