@@ -554,6 +554,18 @@ dust_status dust_noise_fill(dust_noise nz, uint32_t stream_id, int t0, int n_tok
                        "dust_noise_fill");
 }
 
+dust_status dust_noise_sum(dust_noise nz, int T, int d, float* out, void* stream) {
+    DUST_REQUIRE(nz.draw_count > 0, DUST_ERR_INVALID_ARG, "draw_count must be > 0");
+    DUST_REQUIRE(static_cast<uint64_t>(nz.draw_begin) + nz.draw_count <= (1ull << 32), DUST_ERR_INVALID_ARG,
+                 "draw_begin + draw_count exceeds 2^32");
+    DUST_REQUIRE(nz.draw_count <= 0x7FFFFFFFu, DUST_ERR_INVALID_ARG, "draw_count must be < 2^31");
+    DUST_REQUIRE(T > 0 && d > 0, DUST_ERR_INVALID_ARG, "T and d must be > 0");
+    DUST_REQUIRE(nz.token_begin <= 0x7FFFFFFFu, DUST_ERR_INVALID_ARG, "token_begin must be < 2^31");
+    DUST_REQUIRE(static_cast<long long>(T) * d < (1ll << 40), DUST_ERR_INVALID_ARG, "T x d too large");
+    DUST_TRY(check_ptr(out, "out"));
+    return cuda_status(dust::launch_noise_sum(nz, T, d, out, as_stream(stream)), "dust_noise_sum");
+}
+
 dust_status dust_box_muller_words(const uint32_t* a, const uint32_t* b, long long n, float* n_even, float* n_odd,
                                   void* stream) {
     DUST_REQUIRE(n > 0, DUST_ERR_INVALID_ARG, "n must be > 0");

@@ -34,6 +34,8 @@ cudaError_t launch_box_muller_words(const uint32_t* a, const uint32_t* b, long l
                                     cudaStream_t stream);
 cudaError_t launch_synth_costs(const float* u, int T, int d_out, const dust_noise& nz,
                                float eps_scale, float* c, cudaStream_t stream);
+// the generator's ceiling (noise_sum.cu): out[t][j] = sum_k a(draw_begin + k, token_begin + t, j)
+cudaError_t launch_noise_sum(const dust_noise& nz, int T, int d, float* out, cudaStream_t stream);
 
 // a6 / a2 on CUDA cores (gemm_simt.cu):
 //   C[m][n] = sum_k A(m, k) B(k, n), C row-major [M][N] with leading dim ldc.

@@ -85,6 +85,7 @@ _SIGS = {
     "dust_cosine": ([_vp, _vp, C.c_longlong, _vp, _vp, _sz, _vp], _i),
     "dust_cosine_workspace": ([], _sz),
     "dust_noise_fill": ([_Noise, _u, _i, _i, _i, _i, _vp, _vp], _i),
+    "dust_noise_sum": ([_Noise, _i, _i, _vp, _vp], _i),
     "dust_box_muller_words": ([_vp, _vp, C.c_longlong, _vp, _vp, _vp], _i),
     "dust_synth_costs": ([_vp, _i, _i, _Noise, _f, _vp, _vp], _i),
     "dust_toy_suffix_losses": ([_vp, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp, _Noise, _vp, _vp,
@@ -404,6 +405,17 @@ def cosine(a: torch.Tensor, b: torch.Tensor) -> torch.Tensor:
 def noise_fill(noise: Noise, t0: int, n_tok: int, j0: int, n_ch: int, stream_id: int = 0, device="cuda"):
     out = torch.empty(noise.draw_count, n_tok, n_ch, dtype=torch.float32, device=device)
     _check(lib().dust_noise_fill(noise.c(), stream_id, t0, n_tok, j0, n_ch, out.data_ptr(), _stream()))
+    return out
+
+
+def noise_sum(noise: Noise, T: int, d: int, out: torch.Tensor | None = None, device="cuda"):
+    """dust_noise_sum, the generator's ceiling: out[t][j] = the sum over the
+    noise's draw range of a(draw, token_begin + t, j), [T][d] fp32."""
+    if out is None:
+        out = torch.empty(T, d, dtype=torch.float32, device=device)
+    elif tuple(out.shape) != (T, d):
+        raise ValueError("out must be [T][d]")
+    _check(lib().dust_noise_sum(noise.c(), T, d, _dev(out, "out", torch.float32), _stream()))
     return out
 
 

@@ -424,7 +424,8 @@ def main():
     stages = step.stage_times(args.steps)
     clocks = clk.summary()
 
-    kernels = kernel_report(step, stages, peaks, clocks)
+    ceiling = noise_ceiling(step, K)
+    kernels = kernel_report(step, stages, peaks, clocks, ceiling)
     dominant = max((k for k in kernels if not k.get("idle")), key=lambda k: k["ms"])
     e2e = None if args.no_e2e else e2e_run(step, args, world)
     # every tcgen05 / fused kernel records a run-out bounded wait in its workspace's status word:
@@ -455,7 +456,9 @@ def main():
             "roofline": {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
             | {"kernel": dominant["name"], "clock_mhz_for_peak": dominant.get("clock_mhz_for_peak"),
                "peak_source": dominant.get("peak_source"),
-               "fma_heavy_pipe": dominant.get("fma_heavy_pipe")},
+               "fma_heavy_pipe": dominant.get("fma_heavy_pipe"),
+               "noise_ceiling_frac": dominant.get("noise_ceiling_frac")},
+            "noise_ceiling": ceiling,
             "kernels": kernels,
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -526,7 +529,42 @@ def traffic_bytes(terms, K, T, d_out):
     return sum(b * counts[u] for b, u in terms)
 
 
-def kernel_report(step, stages, peaks, clocks):
+def noise_ceiling(step, K):
+    """The generator's empirical ceiling on this GPU: dust_noise_sum (every
+    Gaussian regenerated and consumed by one fma, nothing read from HBM) on the
+    step's widest noise shape, min(K, 256) draws, timed with CUDA events after
+    3 warm-up launches.  It overwrites that layer's g buffer, outside the timed
+    region."""
+    import torch
+    dust, w = step.dust, step.w
+    if step.hidden:
+        L = max(step.hidden, key=lambda L: L["hl"].d_out)
+        out, d, layer = L["g"], L["hl"].d_out, L["hl"].layer
+    elif step.head and step.head["Vr"]:
+        out, d, layer = step.head["g"], step.head["Vr"], w.head_layer
+    else:
+        return None
+    kc = min(K, 256)
+    nz = dust.Noise(w.seed, layer, 0, kc, kc, w.sigma)
+    for _ in range(3):
+        dust.noise_sum(nz, w.T, d, out=out)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = 3
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n):
+        dust.noise_sum(nz, w.T, d, out=out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    return {"kernel": "noise_sum_kernel", "gaussians_per_s": kc * w.T * d / (ms / 1e3), "ms": ms,
+            "draws": kc, "tokens": w.T, "channels": d,
+            "what": "the noise generator alone, each Gaussian consumed by one fma; the ALU-bound kernels' "
+                    "noise_ceiling_frac is their elements/s over this"}
+
+
+def kernel_report(step, stages, peaks, clocks, ceiling=None):
     w, T = step.w, step.w.T
     f_peak = peaks["sm_max_mhz"]
     alu_peak = 148 * LANES_PER_SM * f_peak * 1e6 / 1e12          # T lane-slots/s
@@ -562,6 +600,8 @@ def kernel_report(step, stages, peaks, clocks):
                     "gaussians_per_s": float(K) * T * d_out / (ms / 1e3),
                     "gemm_tflops": 2.0 * T * d_in * d_out / (ms / 1e3) / 1e12,
                     "peak_source": "148 SMs x 4 schedulers x 32 lanes x max SM clock"}
+            if ceiling:
+                rec["noise_ceiling_frac"] = rec["gaussians_per_s"] / ceiling["gaussians_per_s"]
         elif kind in ("weight_grad", "logits"):
             fl = 2.0 * T * d_in * d_out
             ach = fl / (ms / 1e3) / 1e12
@@ -588,6 +628,10 @@ def kernel_report(step, stages, peaks, clocks):
                     "peak_source": "148 SMs x 4 schedulers x 32 lanes x max SM clock (one issue slot per lane "
                                    "per clock); work = the specification's operations in their cheapest sm_100 "
                                    "instruction forms"}
+            if ceiling:
+                # elements (Gaussians of the reduction, perturbed logits of the head) per second over the
+                # generator's own ceiling on this GPU
+                rec["noise_ceiling_frac"] = rec["gaussians_per_s"] / ceiling["gaussians_per_s"]
             # the binding datapath's view of the same kernel: the specification's FMA-heavy cycles
             # against one cycle per lane per scheduler; the issue-slot fraction above cannot exceed
             # slots_per_element / heavy_cycles_per_element on sm_100
@@ -695,9 +739,18 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
+CPU_SAMPLE_SECONDS = 15.0
+
+
 def cpu_baseline(w, K):
+    """The oracle on a bounded sample sized for about CPU_SAMPLE_SECONDS of host
+    work: a probe of one token per host thread, then a multiple of the thread
+    count (the oracle runs tokens in parallel) scaled to the target."""
     cores = cpu_cores()
-    n_tok = max(2, min(512, 2 * cores))
+    n0 = max(1, min(w.T, cores))
+    t0, _, _ = oracle_sample(w, K, n0)
+    n_tok = int(n0 * CPU_SAMPLE_SECONDS / max(t0, 1e-3))
+    n_tok = max(n0, min(w.T, 4096, (n_tok // cores) * cores))
     t_s, units, t_full = oracle_sample(w, K, n_tok)
     n_layers = len(w.hidden) + (1 if w.V else 0)
     return {"value": n_layers * K * w.T / t_full, "unit": UNIT, "cores": cores, "kind": "oracle",

@@ -302,6 +302,22 @@ size_t dust_cosine_workspace(void);
 dust_status dust_noise_fill(dust_noise nz, uint32_t stream_id, int t0, int n_tok,
                             int j0, int n_ch, float *out, void *stream);
 
+/* The generator's empirical ceiling, for measurement: the noise of a draw
+ * range summed per token and channel,
+ *   out[t][j] = sum_{k < draw_count} a(seed, layer, draw_begin + k, token_begin + t, j),
+ * with the noise of the per-token, per-draw N(0, I) activation perturbation
+ * (cnblogs Dust explainer, section "信用分配：一次前向，两种奖励").  Each
+ * Gaussian is consumed by one fused multiply-add that also applies the
+ * Box-Muller radius (acc + rho cos, rounded once), and nothing but out touches
+ * HBM, so its Gaussians/s bound every noise consumer of this library.  The sum
+ * runs in fp32 in a fixed order (even draws and odd draws in two partial sums
+ * added at the end); it equals the sum of the binary32 noise values to within
+ * fp32 rounding.  sigma and K_total are not used.  out: [T][d] fp32 (device,
+ * 16-byte aligned), overwritten.  Errors: DUST_ERR_INVALID_ARG for T, d or
+ * draw_count <= 0, draw_count >= 2^31, a draw or token range beyond 2^32 or
+ * token_begin >= 2^31; DUST_ERR_ALIGNMENT; DUST_ERR_CUDA for a launch error. */
+dust_status dust_noise_sum(dust_noise nz, int T, int d, float *out, void *stream);
+
 /* The noise generator's Box-Muller step on caller-given Philox word pairs:
  * (n_even[i], n_odd[i]) = transform(a[i], b[i]).  a, b: [n] uint32; outputs
  * [n] fp32.  For exhaustive bit-exactness checks of the specification. */

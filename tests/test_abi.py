@@ -97,6 +97,12 @@ def test_invalid_sizes_rejected_on_host(L):
     assert status(L.dust_weight_grad(GOOD, 0, GOOD, 7, 16, 8, 8, GOOD, 0, GOOD, 1 << 20, st)) == 1
     assert status(L.dust_weight_grad(GOOD, 0, GOOD, 0, 0, 8, 8, GOOD, 0, GOOD, 1 << 20, st)) == 1
     assert "must" in L.dust_last_error().decode()
+    # noise sum: empty shapes, no draws, token range past 2^31
+    assert status(L.dust_noise_sum(NZ.c(), 0, 8, GOOD, st)) == 1
+    assert status(L.dust_noise_sum(NZ.c(), 16, 0, GOOD, st)) == 1
+    assert status(L.dust_noise_sum(nz0, 16, 8, GOOD, st)) == 1
+    assert status(L.dust_noise_sum(far, 16, 8, GOOD, st)) == 1
+    assert status(L.dust_noise_sum(NZ.c(), 16, 8, None, st)) == 1
 
 
 def test_misaligned_pointers_rejected_on_host(L):
@@ -105,6 +111,7 @@ def test_misaligned_pointers_rejected_on_host(L):
     assert status(L.dust_reward_scan(GOOD, GOOD + 8, 4, 16, GOOD, 1, 0.5, st)) == 3
     assert status(L.dust_layer_estimate(GOOD, 1, 16, 8, GOOD, 1, 0.0, NZ.c(), GOOD + 2, None, 0, None, 0, st)) == 3
     assert status(L.dust_weight_grad(GOOD, 0, GOOD + 4, 1, 16, 8, 8, GOOD, 0, GOOD, 1 << 20, st)) == 3
+    assert status(L.dust_noise_sum(NZ.c(), 16, 8, GOOD + 4, st)) == 3
     assert "aligned" in L.dust_last_error().decode()
 
 

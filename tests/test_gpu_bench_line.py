@@ -1,0 +1,60 @@
+"""bench.py's one JSON line, run as a user runs it, on small workloads: the
+keys the measurement contract names are present and consistent, the device
+status word reads ok, and every ALU-bound kernel carries its fraction of the
+generator's measured ceiling."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+pytestmark = pytest.mark.gpu
+
+
+def run_bench(*args):
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--steps", "2", "--warmup", "3", "--no-cpu-baseline",
+           *args]
+    out = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout[-2000:]
+    return json.loads(lines[0])
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+@pytest.mark.parametrize("workload,draws", [("head_small_fp32", 16), ("hidden_sweep_bf16", 64)])
+def test_bench_line_contract(workload, draws):
+    line = run_bench("--workload", workload, "--draws", str(draws))
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks",
+                "status", "noise_ceiling", "kernels"):
+        assert key in line, key
+    assert line["status"] == "ok"
+    assert line["n_gpus"] == 1 and line["steps"] == 2 and line["warmup"] == 3
+    assert line["config"]["workload"] == workload and line["config"]["draws"] == draws
+    assert line["value"] > 0 and line["gpu_launches"] > 0
+    e2e = line["e2e"]
+    assert e2e["value"] > 0 and e2e["h2d_bytes_per_step"] > 0 and e2e["d2h_bytes_per_step"] > 0
+    roof = line["roofline"]
+    assert roof["bound"] in ("alu", "hbm", "tensor") and 0 < roof["frac"] == pytest.approx(
+        roof["achieved"] / roof["peak"])
+    ceil = line["noise_ceiling"]
+    assert ceil["kernel"] == "noise_sum_kernel" and ceil["gaussians_per_s"] > 0
+    alu = [k for k in line["kernels"] if k.get("bound") == "alu"]
+    assert alu
+    for k in alu:
+        assert k["noise_ceiling_frac"] == pytest.approx(k["gaussians_per_s"] / ceil["gaussians_per_s"])
+        assert 0 < k["noise_ceiling_frac"]
+    if workload == "hidden_sweep_bf16":
+        # the draw reduction is the generator plus one load-free multiply per pair: near the ceiling
+        for k in alu:
+            assert 0.5 < k["noise_ceiling_frac"] < 1.1, k
