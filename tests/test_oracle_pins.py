@@ -126,6 +126,29 @@ def test_estimate_converges_like_inverse_sqrt_K(orc):
     np.testing.assert_allclose(errs, np.sqrt((d + 1) / Ks), rtol=0.15)
 
 
+def test_estimate_observation_noise_raises_the_cosine_constant(orc):
+    """Synthetic linear costs with observation noise, c = sigma <u, a> + eps e
+    (gamma = 0, so r = c): g stays unbiased and, per token,
+    K E||g + u||^2 / ||u||^2 = d + 1 + d (eps / sigma)^2 / ||u||^2
+    (Var g_j = (||u||^2 + u_j^2 + eps^2 / sigma^2) / K), the constant c of the
+    cosine law cos(K) = c_max / sqrt(1 + c / K).  At eps / sigma = 5 the noise
+    term roughly doubles c, so the pin separates it from the noiseless d + 1."""
+    T, d, sigma, eps, K = 64, 24, 0.01, 0.05, 2048
+    u = I.normal((T, d), 1.0, seed=6)
+    draws = np.repeat(np.arange(K), T)
+    toks = np.tile(np.arange(T), K)
+    c = orc.synth_costs(u, 0, 19, sigma, eps, draws, toks).reshape(K, T).astype(np.float32)
+    g = orc.layer_estimate(c, True, d, [0, T], 0.0, 0, 19, 0, K, sigma, np.arange(T))
+    u2 = np.sum(u.astype(np.float64) ** 2, axis=1)
+    c_emp = K * np.sum((g + u) ** 2, axis=1) / u2
+    c_th = d + 1 + d * (eps / sigma) ** 2 / u2
+    assert abs(np.mean(c_emp) / np.mean(c_th) - 1) < 0.10, (np.mean(c_emp), np.mean(c_th))
+    assert np.mean(c_th) > 1.6 * (d + 1)                     # the noise term is what is being pinned
+    # unbiased: the token-mean of g + u is within a few standard errors of zero
+    se = np.sqrt(np.mean(c_th * u2) / K / d)
+    assert np.all(np.abs(np.mean(g + u, axis=0)) < 5 * se / np.sqrt(T))
+
+
 # ------------------------------------------------------------------ a6 weight estimate
 
 def test_weight_grad_input_invariance_autograd(orc):
