@@ -103,16 +103,34 @@ def parse_args():
     return p.parse_args()
 
 
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+
+
 def load_peaks():
+    """Roofline denominators: MEASURED_PEAKS.json where it holds a positive
+    number for a field, else the fallback; `source` says which fields were
+    measured."""
+    peaks = dict(FALLBACK_PEAKS)
+    measured = []
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(path):
+    try:
         with open(path) as f:
             d = json.load(f)
-        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
-                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
-                "sm_max_mhz": d.get("sm_max_mhz", 1965.0), "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0,
-            "source": "fallback"}
+    except (OSError, ValueError):
+        d = {}
+    if not isinstance(d, dict):
+        d = {}
+    for key in FALLBACK_PEAKS:
+        v = d.get(key)
+        if key == "bf16_tflops_sustained" and v is None:
+            v = d.get("bf16_tflops")
+        if isinstance(v, (int, float)) and not isinstance(v, bool) and v > 0:
+            peaks[key] = float(v)
+            measured.append(key)
+    peaks["measured_keys"] = measured
+    peaks["source"] = ("measured" if len(measured) == len(FALLBACK_PEAKS) else
+                       "fallback" if not measured else "measured: " + ", ".join(measured) + "; fallback: others")
+    return peaks
 
 
 # ------------------------------------------------------------------ clocks
@@ -564,6 +582,12 @@ def noise_ceiling(step, K):
                     "noise_ceiling_frac is their elements/s over this"}
 
 
+def peak_source(peaks, key, what):
+    if key in peaks.get("measured_keys", ()):
+        return f"of measured: MEASURED_PEAKS.json {key} ({what})"
+    return f"of fallback: {FALLBACK_PEAKS[key]:g} from the profiling recipe ({what}); MEASURED_PEAKS.json had none"
+
+
 def kernel_report(step, stages, peaks, clocks, ceiling=None):
     w, T = step.w, step.w.T
     f_peak = peaks["sm_max_mhz"]
@@ -588,7 +612,8 @@ def kernel_report(step, stages, peaks, clocks, ceiling=None):
             byts = 8.0 * K * T
             ach = byts / (ms / 1e3) / 1e9
             rec |= {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": ach / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes": byts}
+                    "frac": ach / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes": byts,
+                    "peak_source": peak_source(peaks, "hbm_gbs", "copy bandwidth")}
         elif kind == "fused_estimate_wgrad":
             # ALU-bound like the reduction it contains; the GEMM's flops ride on the tensor pipe alongside
             slots = float(K) * T * d_out * SLOTS_A5
@@ -606,7 +631,10 @@ def kernel_report(step, stages, peaks, clocks, ceiling=None):
             fl = 2.0 * T * d_in * d_out
             ach = fl / (ms / 1e3) / 1e12
             rec |= {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": ach / peaks["bf16_tflops"], "traffic": None, "algorithmic_flops": fl}
+                    "frac": ach / peaks["bf16_tflops"], "traffic": None, "algorithmic_flops": fl,
+                    "peak_source": peak_source(peaks, "bf16_tflops",
+                                               "cuBLAS bf16 GEMM, burst (each GEMM runs under a millisecond "
+                                               "between ALU-bound kernels, at full clock)")}
         else:
             slots_el = SLOTS_HEAD if layer == "head" else SLOTS_A5
             slots = float(K) * T * d_out * slots_el
@@ -643,7 +671,8 @@ def kernel_report(step, stages, peaks, clocks, ceiling=None):
             # and HBM's: the bytes the kernel must move over its time, against the copy bandwidth
             # (small by construction: the noise is regenerated, never read)
             gbs = alg_bytes / (ms / 1e3) / 1e9
-            rec["hbm"] = {"achieved_gbs": gbs, "frac": gbs / peaks["hbm_gbs"]}
+            rec["hbm"] = {"achieved_gbs": gbs, "frac": gbs / peaks["hbm_gbs"],
+                          "peak_source": peak_source(peaks, "hbm_gbs", "copy bandwidth")}
         out.append(rec)
     return out
 

@@ -81,3 +81,20 @@ def test_noise_sum_is_the_reduction_at_unit_rewards(orc):
     ref = -s / (K * sigma)
     err = float((g - ref).abs().max() / ref.abs().max())
     assert err < 1e-5
+
+
+def test_noise_sum_as_benchmarked(orc):
+    """The launch the benchmark times as the generator's ceiling on the scaled
+    workload: 256 draws over 64 x 1024 tokens x 4096 channels (the widest
+    layer), the noise of its layer; 16 sampled tokens against the oracle."""
+    from activation_perturbation_es_b200 import inputs as I
+    w = I.SCALED
+    hl = max(w.hidden, key=lambda h: h.d_out)
+    T, d, K = w.T, hl.d_out, 256
+    nz = dust.Noise(w.seed, hl.layer, 0, K, K, w.sigma)
+    out = dust.noise_sum(nz, T, d)
+    rs = np.random.Generator(np.random.PCG64(21))
+    toks = np.sort(rs.choice(T, 16, replace=False))
+    got = out[torch.from_numpy(toks).cuda()].cpu().numpy().astype(np.float64)
+    s, sabs, _ = oracle_sum(orc, w.seed, hl.layer, 0, K, toks, d)
+    assert np.all(np.abs(got - s) <= (K + 1) * 2.0 ** -24 * sabs + 1e-30)

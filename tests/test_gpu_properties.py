@@ -98,3 +98,16 @@ def test_fused_random_shapes(orc, lengths, d_out, d_in, K, gamma, seed, tb):
     G_ref = oracle_chains.weight_rows(orc, c, False, d_out, off, gamma, nz.seed, 4, 0, K, 0.01, X, np.arange(d_out),
                                       token_begin=tb)
     assert rel_err(G.cpu().numpy(), G_ref) < FP32_TOL
+
+
+@settings(**dict(SETTINGS, max_examples=40))
+@given(T=st.integers(1, 70), d=st.integers(1, 300), K=st.integers(1, 40), draw0=st.integers(0, 1 << 20),
+       seed=st.integers(0, 2**32 - 1), tb=st.integers(0, 1 << 30))
+def test_noise_sum_random_shapes(orc, T, d, K, draw0, seed, tb):
+    """The ceiling kernel on random shapes: within the fp32 bound of a
+    fixed-order sum, |out - sum a| <= (K + 1) 2^-24 sum |a|, of the oracle's
+    noise summed in float64."""
+    nz = dust.Noise(seed, 4, draw0, K, K, 1e-2, token_begin=tb)
+    got = dust.noise_sum(nz, T, d).cpu().numpy().astype(np.float64)
+    a = orc.noise_block(seed, 4, draw0, K, np.arange(T) + tb, 0, d).astype(np.float64)
+    assert np.all(np.abs(got - a.sum(axis=0)) <= (K + 1) * 2.0 ** -24 * np.abs(a).sum(axis=0) + 1e-30)
