@@ -21,6 +21,15 @@ namespace dust {
 
 namespace {
 
+// M1 d stepped to M1 (d + 1) as one plain 64-bit add: the same value as
+// next_draw's carry chain, left to the compiler's choice of form, which runs
+// this kernel about 1% faster (the draw reduction is unchanged by it).
+__device__ __forceinline__ void next_draw_u64(DrawProduct& p) {
+    const unsigned long long v = ((static_cast<unsigned long long>(p.hi) << 32) | p.lo) + kPhiloxM1;
+    p.lo = static_cast<uint32_t>(v);
+    p.hi = static_cast<uint32_t>(v >> 32);
+}
+
 // xz += rho (cos) and yw += rho (sin) for the 4 channels of one Philox call,
 // as two packed lanes (channels (4q, 4q+2) and (4q+1, 4q+3))
 __device__ __forceinline__ void sum_quad_after_round1(float2& xz, float2& yw, uint4 c1, uint32_t seed,
@@ -45,19 +54,19 @@ noise_sum_kernel(int T, int d, int nq, uint32_t seed, uint32_t layer, uint32_t d
         int k = 0;
         for (; k + 4 <= nd; k += 4) {
             sum_quad_after_round1(xz0, yw0, philox_round1_state(dp, tok, seed, rq), seed, layer);
-            next_draw(dp);
+            next_draw_u64(dp);
             sum_quad_after_round1(xz1, yw1, philox_round1_state(dp, tok, seed, rq), seed, layer);
-            next_draw(dp);
+            next_draw_u64(dp);
             sum_quad_after_round1(xz0, yw0, philox_round1_state(dp, tok, seed, rq), seed, layer);
-            next_draw(dp);
+            next_draw_u64(dp);
             sum_quad_after_round1(xz1, yw1, philox_round1_state(dp, tok, seed, rq), seed, layer);
-            next_draw(dp);
+            next_draw_u64(dp);
         }
         for (; k + 2 <= nd; k += 2) {
             sum_quad_after_round1(xz0, yw0, philox_round1_state(dp, tok, seed, rq), seed, layer);
-            next_draw(dp);
+            next_draw_u64(dp);
             sum_quad_after_round1(xz1, yw1, philox_round1_state(dp, tok, seed, rq), seed, layer);
-            next_draw(dp);
+            next_draw_u64(dp);
         }
         if (k < nd) sum_quad_after_round1(xz0, yw0, philox_round1_state(dp, tok, seed, rq), seed, layer);
         const float v[4] = {xz0.x + xz1.x, yw0.x + yw1.x, xz0.y + xz1.y, yw0.y + yw1.y};
