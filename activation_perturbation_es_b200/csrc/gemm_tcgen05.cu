@@ -19,9 +19,15 @@
 //           and frees TMEM: two BN-column fp32 accumulators (2 BN columns), so
 //           that unit i's epilogue overlaps unit i+1's main loop;
 //   warps 2-9: epilogue, two warps per TMEM lane quarter taking alternate
-//           32-column blocks: tcgen05.ld of the warp's 32 TMEM lanes (rows),
-//           an xor-swizzled 32 x 32 shared-memory transpose, then row-segment
-//           fp32 stores; the warps release the accumulator buffer afterwards.
+//           32-column blocks: tcgen05.ld of the warp's 32 TMEM lanes (rows)
+//           into registers, then the block into shared memory in the TMA's
+//           128-byte-swizzled layout (eight conflict-free 16-byte stores per
+//           lane) and one TMA store of the 32 x 32 block (C, or the split's
+//           partial slab through a 3-D map); the tensor map clips ragged edges.
+//           When C is accumulated into, or its row pitch is not a multiple of
+//           16 bytes, the block goes through an xor-swizzled shared transpose to
+//           row-segment fp32 stores instead.  The warps release the accumulator
+//           buffer once its columns are in registers.
 // Split over k writes fp32 partial tiles that a second kernel sums in a fixed
 // order (deterministic).  Every mbarrier wait is bounded: when a bound runs
 // out the role records the workspace status word, raises the CTA's abort flag
@@ -29,6 +35,7 @@
 // (bounded too), frees TMEM and returns.
 #include <cuda.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -91,6 +98,10 @@ __device__ __forceinline__ Unit unit_of(int u, int tiles_m, int tiles_n, int BN,
 }
 
 constexpr int kEpiWarps = 8;                          // two per TMEM lane quarter
+// how the epilogue writes a 32 x 32 block: generic stores after a shared
+// transpose; a TMA store into C ([M][N], 2-D map); a TMA store into the
+// split's partial slab ([splits][M][N], 3-D map)
+constexpr int kStoreGeneric = 0, kStoreC = 1, kStorePartial = 2;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;     // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 
 // Persistent, warp-specialised: every CTA walks the work units (tile, k
@@ -100,9 +111,10 @@ constexpr int kGemmThreads = 64 + 32 * kEpiWarps;     // warp 0 TMA, warp 1 MMA,
 // atoms of 64 K rows each); B likewise with BN rows / BN/64 atoms.
 template <int BN, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, int M, int N,
-               int K, int k_per_split, int splits, float* __restrict__ C, int ldc, int accumulate,
-               float* __restrict__ partial, uint32_t* __restrict__ status) {
+gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+               const __grid_constant__ CUtensorMap map_c, int store_mode, int M, int N, int K, int k_per_split,
+               int splits, float* __restrict__ C, int ldc, int accumulate, float* __restrict__ partial,
+               uint32_t* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     using S = Smem<BN>;
@@ -261,6 +273,25 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] = 0.0f;
                 }
+                if (store_mode != kStoreGeneric) {
+                    // the previous block's store has finished reading the buffer
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+                    // row `lane` of the block: 16-byte chunk g at chunk position g ^ (row mod 8)
+                    float4* rowp = reinterpret_cast<float4*>(tile + lane * 32);
+#pragma unroll
+                    for (int g = 0; g < 8; ++g)
+                        rowp[g ^ (lane & 7)] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+                    fence_proxy_async_shared();
+                    __syncwarp();
+                    const int col0 = w.n0 + c0;
+                    if (lane == 0 && row0 < M && col0 < N) {
+                        if (store_mode == kStoreC) tma_store_2d(&map_c, tile, col0, row0);
+                        else tma_store_3d(&map_c, tile, col0, row0, split);
+                        bulk_commit();
+                    }
+                    continue;
+                }
 #pragma unroll
                 for (int i = 0; i < 32; ++i) tile[lane * 32 + (i ^ lane)] = v[i];
                 __syncwarp();
@@ -281,6 +312,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             __syncwarp();
             if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&tempty[buf])) : "memory");
         }
+        // the block stores this warp issued have completed before the CTA's
+        // shared memory goes away
+        if (store_mode != kStoreGeneric && lane == 0) bulk_wait_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -329,6 +363,24 @@ bool make_map(CUtensorMap* map, const void* base, int inner, int outer, int ld, 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 output of the epilogue's TMA stores: [outer2][outer1][inner] with row
+// pitch `ld` floats (outer2 = 1 gives the 2-D map of C), box {32, 32, 1},
+// 128-byte swizzle (one 32-float row is one 128-byte swizzle row).
+bool make_store_map(CUtensorMap* map, float* base, int inner, int outer1, int ld, int outer2) {
+    EncodeTiled enc = encode_fn();
+    if (enc == nullptr || (reinterpret_cast<uintptr_t>(base) & 15u) != 0 || (ld & 3) != 0) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer1),
+                                static_cast<cuuint64_t>(outer2)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * 4,
+                                   static_cast<cuuint64_t>(ld) * 4 * static_cast<cuuint64_t>(outer1)};
+    const cuuint32_t box[3] = {32u, 32u, 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    const cuuint32_t rank = outer2 > 1 ? 3u : 2u;
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, rank, base, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int pick_bn(int N) { return N >= 256 ? 256 : (N > 64 ? 128 : 64); }
 
 int sm_count() {
@@ -344,8 +396,9 @@ int sm_count() {
 }
 
 template <int BN, bool A_MN, bool B_MN>
-cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int K, int kps, int splits,
-                     float* C, int ldc, int accumulate, float* partial, uint32_t* status, cudaStream_t st) {
+cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, int store_mode, int M,
+                     int N, int K, int kps, int splits, float* C, int ldc, int accumulate, float* partial,
+                     uint32_t* status, cudaStream_t st) {
     auto kern = gemm_tc_kernel<BN, A_MN, B_MN>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
@@ -357,18 +410,22 @@ cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N,
     const int per_sm = Smem<BN>::kBytes * 2 <= 227 * 1024 ? 2 : 1;   // TMEM: 2 x 2 BN <= 512 columns for BN <= 128
     const long long grid = units < static_cast<long long>(sm_count()) * per_sm ? units : sm_count() * per_sm;
     kern<<<static_cast<unsigned>(grid), kGemmThreads, Smem<BN>::kBytes, st>>>(
-        ma, mb, M, N, K, kps, splits, C, ldc, accumulate, splits > 1 ? partial : nullptr, status);
+        ma, mb, mc, store_mode, M, N, K, kps, splits, C, ldc, accumulate, splits > 1 ? partial : nullptr, status);
     return cudaGetLastError();
 }
 
 template <bool A_MN, bool B_MN>
-cudaError_t launch_bn(int bn, const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int K, int kps, int splits,
-                      float* C, int ldc, int accumulate, float* partial, uint32_t* status, cudaStream_t st) {
+cudaError_t launch_bn(int bn, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, int store_mode,
+                      int M, int N, int K, int kps, int splits, float* C, int ldc, int accumulate, float* partial,
+                      uint32_t* status, cudaStream_t st) {
+#define DUST_GEMM_BN(BN_)                                                                                        \
+    launch_t<BN_, A_MN, B_MN>(ma, mb, mc, store_mode, M, N, K, kps, splits, C, ldc, accumulate, partial, status, st)
     switch (bn) {
-        case 256: return launch_t<256, A_MN, B_MN>(ma, mb, M, N, K, kps, splits, C, ldc, accumulate, partial, status, st);
-        case 128: return launch_t<128, A_MN, B_MN>(ma, mb, M, N, K, kps, splits, C, ldc, accumulate, partial, status, st);
-        default: return launch_t<64, A_MN, B_MN>(ma, mb, M, N, K, kps, splits, C, ldc, accumulate, partial, status, st);
+        case 256: return DUST_GEMM_BN(256);
+        case 128: return DUST_GEMM_BN(128);
+        default: return DUST_GEMM_BN(64);
     }
+#undef DUST_GEMM_BN
 }
 
 }  // namespace
@@ -425,15 +482,29 @@ cudaError_t launch_gemm_tc(const void* A, bool a_kmajor, int lda, const void* B,
     const bool okB = b_kmajor ? make_map(&mb, B, K, N, ldb, bn) : make_map(&mb, B, N, K, ldb, kBK);
     if (!okA || !okB) return cudaErrorInvalidValue;
     const int kps = static_cast<int>(ceil_div(ceil_div(K, splits), kBK) * kBK);
+    // the epilogue's store: TMA into the split-K slabs or into C where the
+    // tensor map can describe them; generic stores otherwise (and whenever C
+    // is accumulated into, which needs a read)
+    CUtensorMap mc;
+    std::memset(&mc, 0, sizeof(mc));
+    int store_mode = kStoreGeneric;
+    if (splits > 1) {
+        if (make_store_map(&mc, partial, N, M, N, splits)) store_mode = kStorePartial;
+    } else if (!accumulate) {
+        if (make_store_map(&mc, C, N, M, ldc, 1)) store_mode = kStoreC;
+    }
     cudaError_t e;
+#define DUST_GEMM_MAJOR(AMN_, BMN_)                                                                              \
+    launch_bn<AMN_, BMN_>(bn, ma, mb, mc, store_mode, M, N, K, kps, splits, C, ldc, accumulate, partial, status, stream)
     if (!a_kmajor && !b_kmajor)
-        e = launch_bn<true, true>(bn, ma, mb, M, N, K, kps, splits, C, ldc, accumulate, partial, status, stream);
+        e = DUST_GEMM_MAJOR(true, true);
     else if (a_kmajor && b_kmajor)
-        e = launch_bn<false, false>(bn, ma, mb, M, N, K, kps, splits, C, ldc, accumulate, partial, status, stream);
+        e = DUST_GEMM_MAJOR(false, false);
     else if (a_kmajor)
-        e = launch_bn<false, true>(bn, ma, mb, M, N, K, kps, splits, C, ldc, accumulate, partial, status, stream);
+        e = DUST_GEMM_MAJOR(false, true);
     else
-        e = launch_bn<true, false>(bn, ma, mb, M, N, K, kps, splits, C, ldc, accumulate, partial, status, stream);
+        e = DUST_GEMM_MAJOR(true, false);
+#undef DUST_GEMM_MAJOR
     if (e != cudaSuccess || splits == 1) return e;
     return launch_splitk_reduce(partial, splits, M, N, C, ldc, accumulate, stream);
 }
