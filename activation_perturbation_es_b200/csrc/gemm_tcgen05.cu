@@ -24,9 +24,10 @@
 //           128-byte-swizzled layout (eight conflict-free 16-byte stores per
 //           lane) and one TMA store of the 32 x 32 block (C, or the split's
 //           partial slab through a 3-D map); the tensor map clips ragged edges.
-//           When C is accumulated into, or its row pitch is not a multiple of
-//           16 bytes, the block goes through an xor-swizzled shared transpose to
-//           row-segment fp32 stores instead.  The warps release the accumulator
+//           When C is accumulated into, the TMA adds the block into C (one
+//           fp32 addition per element, as C + x).  When C's row pitch is not a
+//           multiple of 16 bytes, the block goes through an xor-swizzled shared
+//           transpose to row-segment fp32 stores instead.  The warps release the accumulator
 //           buffer once its columns are in registers.
 // Split over k writes fp32 partial tiles that a second kernel sums in a fixed
 // order (deterministic).  Every mbarrier wait is bounded: when a bound runs
@@ -100,8 +101,8 @@ __device__ __forceinline__ Unit unit_of(int u, int tiles_m, int tiles_n, int BN,
 constexpr int kEpiWarps = 8;                          // two per TMEM lane quarter
 // how the epilogue writes a 32 x 32 block: generic stores after a shared
 // transpose; a TMA store into C ([M][N], 2-D map); a TMA store into the
-// split's partial slab ([splits][M][N], 3-D map)
-constexpr int kStoreGeneric = 0, kStoreC = 1, kStorePartial = 2;
+// split's partial slab ([splits][M][N], 3-D map); a TMA reduce-add into C
+constexpr int kStoreGeneric = 0, kStoreC = 1, kStorePartial = 2, kAddC = 3;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;     // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 
 // Persistent, warp-specialised: every CTA walks the work units (tile, k
@@ -287,6 +288,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
                     const int col0 = w.n0 + c0;
                     if (lane == 0 && row0 < M && col0 < N) {
                         if (store_mode == kStoreC) tma_store_2d(&map_c, tile, col0, row0);
+                        else if (store_mode == kAddC) tma_reduce_add_2d(&map_c, tile, col0, row0);
                         else tma_store_3d(&map_c, tile, col0, row0, split);
                         bulk_commit();
                     }
@@ -482,16 +484,16 @@ cudaError_t launch_gemm_tc(const void* A, bool a_kmajor, int lda, const void* B,
     const bool okB = b_kmajor ? make_map(&mb, B, K, N, ldb, bn) : make_map(&mb, B, N, K, ldb, kBK);
     if (!okA || !okB) return cudaErrorInvalidValue;
     const int kps = static_cast<int>(ceil_div(ceil_div(K, splits), kBK) * kBK);
-    // the epilogue's store: TMA into the split-K slabs or into C where the
-    // tensor map can describe them; generic stores otherwise (and whenever C
-    // is accumulated into, which needs a read)
+    // the epilogue's store: TMA into the split-K slabs, or into C (a store, or
+    // a reduce-add when C is accumulated into) where the tensor map can
+    // describe them; generic stores otherwise
     CUtensorMap mc;
     std::memset(&mc, 0, sizeof(mc));
     int store_mode = kStoreGeneric;
     if (splits > 1) {
         if (make_store_map(&mc, partial, N, M, N, splits)) store_mode = kStorePartial;
-    } else if (!accumulate) {
-        if (make_store_map(&mc, C, N, M, ldc, 1)) store_mode = kStoreC;
+    } else if (make_store_map(&mc, C, N, M, ldc, 1)) {
+        store_mode = accumulate ? kAddC : kStoreC;
     }
     cudaError_t e;
 #define DUST_GEMM_MAJOR(AMN_, BMN_)                                                                              \
