@@ -257,9 +257,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             tc_fence_after();
             have = w.nk > 0;
             const int split = u / (tiles_m * tiles_n);
-            // Each 32 x 32 block (this warp's 32 rows x 32 columns) goes through a
-            // padded shared tile so that the global stores are row segments:
-            // after the transpose lane l holds column c0 + l of every row.
+            // Each 32 x 32 block (this warp's 32 rows x 32 columns) goes through the
+            // warp's 4 KB shared buffer: in the TMA's swizzled layout for a bulk
+            // store, or xor-swizzled and transposed (lane l then holds column
+            // c0 + l of every row) for row-segment stores.
             float* tile = epi + (warp - 2) * (32 * 32);
             const int row0 = w.m0 + quarter * 32;
             float* base = partial != nullptr ? partial + static_cast<size_t>(split) * M * N : C;
