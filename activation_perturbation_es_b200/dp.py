@@ -49,6 +49,13 @@ def chunk_range(n_chunks: int, world: int, rank: int) -> tuple[int, int]:
     return b, e - b
 
 
+def _host_staged(group, t: torch.Tensor) -> bool:
+    """A gloo process group exchanges device tensors through host copies (the
+    plumbing of a multi-process run on CPU ranks or on one shared GPU)."""
+    import torch.distributed as dist
+    return t.is_cuda and dist.get_backend(group) == "gloo"
+
+
 def allgather_rows(local: torch.Tensor, counts, group=None) -> torch.Tensor:
     """Concatenate every rank's row block (rank order): local is [counts[rank]][...];
     blocks are padded to the largest count for the collective and trimmed after."""
@@ -62,8 +69,14 @@ def allgather_rows(local: torch.Tensor, counts, group=None) -> torch.Tensor:
     rest = tuple(local.shape[1:])
     pad = torch.zeros((most,) + rest, dtype=local.dtype, device=local.device)
     pad[:local.shape[0]].copy_(local)
-    parts = [torch.empty_like(pad) for _ in range(world)]
-    dist.all_gather(parts, pad, group=group)
+    if _host_staged(group, pad):
+        host = pad.cpu()
+        parts = [torch.empty_like(host) for _ in range(world)]
+        dist.all_gather(parts, host, group=group)
+        parts = [p.to(local.device) for p in parts]
+    else:
+        parts = [torch.empty_like(pad) for _ in range(world)]
+        dist.all_gather(parts, pad, group=group)
     return torch.cat([p[:n] for p, n in zip(parts, counts)])
 
 
@@ -79,7 +92,12 @@ def allreduce_sum_(tensors, group=None) -> None:
         by_dtype.setdefault(t.dtype, []).append(t)
     for ts in by_dtype.values():
         flat = torch.cat([t.reshape(-1) for t in ts])
-        dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+        if _host_staged(group, flat):
+            host = flat.cpu()
+            dist.all_reduce(host, op=dist.ReduceOp.SUM, group=group)
+            flat.copy_(host)
+        else:
+            dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
         off = 0
         for t in ts:
             n = t.numel()

@@ -189,6 +189,16 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ distributed plumbing
+def dist_backend():
+    """NCCL, one rank per GPU; DUST_BENCH_DIST_BACKEND=gloo runs the same
+    multi-rank flow with host-side collectives, which lets ranks share a GPU
+    (no kernel of this library waits on another rank)."""
+    b = os.environ.get("DUST_BENCH_DIST_BACKEND", "nccl")
+    if b not in ("nccl", "gloo"):
+        sys.exit(f"bench: DUST_BENCH_DIST_BACKEND must be nccl or gloo, not {b!r}")
+    return b
+
+
 def dist_setup(args):
     import torch
     import torch.distributed as dist
@@ -197,9 +207,13 @@ def dist_setup(args):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if dist_backend() == "gloo":
+            torch.cuda.set_device(local % torch.cuda.device_count())
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=300))
+        else:
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
     return world, rank, local
@@ -216,7 +230,7 @@ def max_over_ranks(x, world):
     import torch.distributed as dist
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device="cpu" if dist.get_backend() == "gloo" else "cuda")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -467,6 +481,7 @@ def main():
                        "hidden": [[h.d_in, h.d_out] for h in w.hidden],
                        "head": {"d": w.head_d, "V": w.V, "Vc": w.Vc} if w.V else None,
                        "parallelism": step.parallelism(), "shard": step.shard,
+                       "dist_backend": dist_backend() if world > 1 else None,
                        "l2": "inputs larger than L2 (126 MB); no flush",
                        "fused_estimate_wgrad": bool(args.fused),
                        "arithmetic": "f32 noise, cross entropy and reductions; bf16 GEMM operands with f32 "
