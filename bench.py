@@ -235,6 +235,47 @@ def max_over_ranks(x, world):
     return float(t.item())
 
 
+# ------------------------------------------------------------------ the workload as both arms name it
+def parallelism(shard, world):
+    return {"sequences": f"dp{world}", "draws": f"draws{world}", "vocab": f"draws{world}+head_vocab{world}"}[shard]
+
+
+def workload_config(w, K, world, shard, fused):
+    """The `config` object of the line, the same for this library's arm and the
+    reference arm: the workload, its population and how N ranks split it."""
+    return {"workload": w.name, "tokens_per_rank": w.T, "n_seq": w.n_seq, "seq_len": w.seq_len,
+            "draws": K, "sigma": w.sigma, "gamma_hidden": w.gamma,
+            "hidden": [[h.d_in, h.d_out] for h in w.hidden],
+            "head": {"d": w.head_d, "V": w.V, "Vc": w.Vc} if w.V else None,
+            "parallelism": parallelism(shard, world), "shard": shard,
+            "dist_backend": dist_backend() if world > 1 else None,
+            "l2": l2_statement(w, K),
+            "fused_estimate_wgrad": bool(fused)}
+
+
+L2_BYTES = 126 * 2**20
+
+
+def step_bytes(w, K):
+    """Bytes one step streams through HBM on one rank: each hidden layer's costs
+    (read by the scan, rewards written and read), layer input and g (fp32 and
+    bf16); the head's logits, g and operands."""
+    b = 0
+    for h in w.hidden:
+        b += 3 * 4 * K * w.T + 2 * w.T * h.d_in + 6 * w.T * h.d_out
+    if w.V:
+        b += 4 * w.T * w.V + 6 * w.T * w.V + 2 * (w.T + w.V) * w.head_d
+    return b
+
+
+def l2_statement(w, K):
+    mb = step_bytes(w, K) / 2**20
+    if step_bytes(w, K) > L2_BYTES:
+        return f"inputs larger than L2 ({mb:.0f} MB per step against 126 MB); no flush"
+    return (f"inputs smaller than L2 ({mb:.1f} MB per step against 126 MB): a warm-L2 small case, not a "
+            f"configuration for headline numbers")
+
+
 # ------------------------------------------------------------------ the step
 class Step:
     """Device-resident buffers and the sequence of C-ABI calls of one step on
@@ -325,8 +366,7 @@ class Step:
         return "weak" if self.shard == "sequences" else "strong"
 
     def parallelism(self):
-        return {"sequences": f"dp{self.world}", "draws": f"draws{self.world}",
-                "vocab": f"draws{self.world}+head_vocab{self.world}"}[self.shard]
+        return parallelism(self.shard, self.world)
 
     def make_events(self, n_steps):
         ev = self.torch.cuda.Event
@@ -475,17 +515,10 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": step.scaling(),
             "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic (seeded; inputs > L2, no flush needed)",
-            "config": {"workload": w.name, "tokens_per_rank": w.T, "n_seq": w.n_seq, "seq_len": w.seq_len,
-                       "draws": K, "sigma": w.sigma, "gamma_hidden": w.gamma,
-                       "hidden": [[h.d_in, h.d_out] for h in w.hidden],
-                       "head": {"d": w.head_d, "V": w.V, "Vc": w.Vc} if w.V else None,
-                       "parallelism": step.parallelism(), "shard": step.shard,
-                       "dist_backend": dist_backend() if world > 1 else None,
-                       "l2": "inputs larger than L2 (126 MB); no flush",
-                       "fused_estimate_wgrad": bool(args.fused),
-                       "arithmetic": "f32 noise, cross entropy and reductions; bf16 GEMM operands with f32 "
-                                     "accumulation in TMEM (tcgen05)"},
+            "data": "synthetic (seeded)",
+            "config": workload_config(w, K, world, args.shard, args.fused),
+            "arithmetic": "f32 noise, cross entropy and reductions; bf16 GEMM operands with f32 accumulation in "
+                          "TMEM (tcgen05)",
             "roofline": {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
             | {"kernel": dominant["name"], "clock_mhz_for_peak": dominant.get("clock_mhz_for_peak"),
                "peak_source": dominant.get("peak_source"),
@@ -827,7 +860,8 @@ def reference_arm(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_full / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
-            "data": "synthetic", "config": {"workload": w.name, "draws": K, "tokens_per_rank": w.T},
+            "data": "synthetic", "config": workload_config(w, K, world, args.shard, args.fused),
+            "arithmetic": "the oracle: float64 accumulation, binary32 noise",
             "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": cores,
                              "sample": f"{n_tok} tokens per layer per step, all draws and channels, "
                                        f"extrapolated linearly in tokens"},

@@ -46,3 +46,26 @@ def test_partial_or_invalid_fields_fall_back_one_by_one(tmp_path, monkeypatch):
 def test_malformed_file_uses_the_fallback(tmp_path, monkeypatch):
     assert peaks_from(tmp_path, monkeypatch, "{not json")["source"] == "fallback"
     assert peaks_from(tmp_path, monkeypatch, "[1, 2]")["source"] == "fallback"
+
+
+def test_l2_statement_follows_the_working_set():
+    from activation_perturbation_es_b200 import inputs as I
+    assert bench.l2_statement(I.SCALED, I.SCALED.K).startswith("inputs larger than L2")
+    assert bench.l2_statement(I.HEAD_PAGES, 64).startswith("inputs larger than L2")
+    assert bench.l2_statement(I.HEAD_SMALL, 16).startswith("inputs smaller than L2")
+    # the scaled step streams about 11 GB: the costs and rewards of both hidden layers dominate
+    assert 10e9 < bench.step_bytes(I.SCALED, I.SCALED.K) < 13e9
+
+
+def test_reference_arm_names_the_same_workload_config():
+    """The reference arm's line carries the library arm's config object, so the
+    two lines compare as the same configuration."""
+    import subprocess
+    from activation_perturbation_es_b200 import inputs as I
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                          "head_small_fp32", "--steps", "1", "--warmup", "1"], cwd=ROOT, capture_output=True,
+                         text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads([ln for ln in out.stdout.splitlines() if ln.startswith("{")][-1])
+    assert line["impl"] == "reference"
+    assert line["config"] == bench.workload_config(I.HEAD_SMALL, 16, 1, "sequences", False)
