@@ -181,8 +181,10 @@ def test_weight_grad_f32(orc, T, d_in, d_out):
 
 
 @pytest.mark.parametrize("T,d_in,d_out", [(256, 64, 128), (1000, 48, 32), (16384, 512, 512), (2048, 2048, 512),
-                                          (16384, 512, 4096)])
+                                          (16384, 512, 4096), (16384, 520, 136)])
 def test_weight_grad_bf16(orc, T, d_in, d_out):
+    """(16384, 520, 136) splits k, and its tiles are ragged in both output
+    dimensions: the split slabs' TMA stores are clipped by the 3-D map."""
     g = I.bf16_round(I.normal((T, d_out), 1.0, seed=T))
     X = I.bf16_round(I.normal((T, d_in), 1.0, seed=T + 1))
     G = host(dust.weight_grad(cu(g, torch.bfloat16), cu(X, torch.bfloat16)))
@@ -222,8 +224,10 @@ def test_weight_grad_mixed_dtypes(orc, g_bf16, T, d_in, d_out):
     assert rel_err(host(G), orc.weight_grad(g, X) + G0.astype(np.float64)) < 1e-5
 
 
-@pytest.mark.parametrize("T,d_in,V", [(1000, 64, 520), (256, 1024, 4096)])
+@pytest.mark.parametrize("T,d_in,V", [(1000, 64, 520), (256, 1024, 4096), (1000, 64, 522)])
 def test_logits_bf16_tensor_cores(orc, T, d_in, V):
+    """V = 522: a row pitch that is not a multiple of 16 bytes, which the
+    epilogue writes with row stores instead of TMA stores."""
     X = I.bf16_round(I.normal((T, d_in), 1.0, seed=T))
     W = I.bf16_round(I.normal((V, d_in), 1.0 / np.sqrt(d_in), seed=V))
     Z = dust.logits(cu(X, torch.bfloat16), cu(W, torch.bfloat16))
