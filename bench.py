@@ -728,52 +728,78 @@ def kernel_report(step, stages, peaks, clocks, ceiling=None):
 # ------------------------------------------------------------------ end to end
 def e2e_run(step, args, world):
     """Same metric through the public API with host buffers: every step copies its
-    inputs from pinned host memory and reads the weight estimates back.  The
-    copies of layer l + 1 run on a copy stream while layer l computes; events
-    order each layer's compute after its own inputs have landed."""
+    inputs from pinned host memory and reads the weight estimates back, inside
+    the timed region.  The device inputs are double-buffered: while step i
+    computes on one set, a copy stream fills the other with step i + 1's inputs
+    (once step i - 1 has finished reading it), and each layer's compute waits on
+    an event recorded after its own inputs have landed."""
     import torch
-    groups = []        # per layer: [(device tensor, pinned host copy)], in compute order
+    # per layer, in compute order: [(container, key, pinned host copy)]
+    groups = []
     for L in step.hidden:
-        groups.append([(L["c"], L["c"].cpu().pin_memory()), (L["X"], L["X"].cpu().pin_memory())])
+        groups.append([(L, "c", L["c"].cpu().pin_memory()), (L, "X", L["X"].cpu().pin_memory())])
     if step.head:
-        groups.append([(step.head[k], step.head[k].cpu().pin_memory()) for k in ("X", "W", "y")])
+        groups.append([(step.head, k, step.head[k].cpu().pin_memory()) for k in ("X", "W", "y")])
+    # two device sets of the inputs: the step's own tensors and a second copy of each
+    sets = [[[cont[key] for cont, key, _ in g] for g in groups],
+            [[torch.empty_like(cont[key]) for cont, key, _ in g] for g in groups]]
     outs = [L["G"] for L in step.hidden] + ([step.head["G"]] if step.head else [])
     outs_h = [o.cpu().pin_memory() for o in outs]
-    h2d = sum(h.numel() * h.element_size() for g in groups for _, h in g)
+    h2d = sum(h.numel() * h.element_size() for g in groups for _, _, h in g)
     d2h = sum(o.numel() * o.element_size() for o in outs_h)
     compute = torch.cuda.current_stream()
     copy = torch.cuda.Stream()
+    freed = [torch.cuda.Event(), torch.cuda.Event()]     # set k no longer read by the compute stream
+    for ev in freed:
+        ev.record(compute)
 
-    def one():
+    def bind(k):
+        for g, devs in zip(groups, sets[k]):
+            for (cont, key, _), d in zip(g, devs):
+                cont[key] = d
+
+    def copy_in(k):
+        copy.wait_event(freed[k])
         ready = []
-        copy.wait_stream(compute)                      # previous step's kernels are done with the buffers
         with torch.cuda.stream(copy):
-            for g in groups:
-                for dev_t, host_t in g:
-                    dev_t.copy_(host_t, non_blocking=True)
+            for g, devs in zip(groups, sets[k]):
+                for (_, _, host), d in zip(g, devs):
+                    d.copy_(host, non_blocking=True)
                 ev = torch.cuda.Event()
                 ev.record(copy)
                 ready.append(ev)
-        step.run_overlapped(ready)
-        for o, oh in zip(outs, outs_h):
-            oh.copy_(o, non_blocking=True)
+        return ready
 
-    one()
+    def run(n):
+        copy.wait_stream(compute)                          # nothing is copied before the region starts
+        ready = copy_in(0)
+        for i in range(n):
+            nxt = copy_in((i + 1) % 2) if i + 1 < n else None
+            bind(i % 2)
+            step.run_overlapped(ready)
+            freed[i % 2].record(compute)
+            for o, oh in zip(outs, outs_h):
+                oh.copy_(o, non_blocking=True)
+            ready = nxt
+
+    run(2)
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n = max(1, min(args.steps, 3))
     barrier(world)
     torch.cuda.synchronize()
     t0.record(compute)
-    for _ in range(n):
-        one()
+    run(n)
     t1.record(compute)
     torch.cuda.synchronize()
     barrier(world)
+    bind(0)
+    del sets
     ms = max_over_ranks(t0.elapsed_time(t1), world) / n
     return {"value": step.total_units() / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": n,
-            "copies": "pinned host -> device on a copy stream, overlapped with the previous layer's compute"}
+            "copies": "pinned host -> device on a copy stream into double-buffered inputs: step i + 1's copies "
+                      "overlap step i's compute, layer by layer"}
 
 
 # ------------------------------------------------------------------ CPU oracle

@@ -58,3 +58,29 @@ def test_bench_line_contract(workload, draws):
         # the draw reduction is the generator plus one load-free multiply per pair: near the ceiling
         for k in alu:
             assert 0.5 < k["noise_ceiling_frac"] < 1.1, k
+
+
+def test_end_to_end_leg_computes_the_same_step():
+    """The end-to-end leg (double-buffered device inputs, copied from pinned
+    host memory while the previous step computes) leaves every weight estimate
+    equal, bit for bit, to the device-resident step's."""
+    import sys as _sys
+    _sys.path.insert(0, ROOT)
+    import argparse
+    import bench
+    from activation_perturbation_es_b200 import inputs as I
+    w = I.HIDDEN_SWEEP
+    step = bench.Step(w, 64, rank=0, world=1)
+    step.run()
+    torch.cuda.synchronize()
+    ref = [L["G"].clone() for L in step.hidden]
+    out = bench.e2e_run(step, argparse.Namespace(steps=3), 1)
+    torch.cuda.synchronize()
+    assert out["value"] > 0 and out["h2d_bytes_per_step"] > 0
+    for L, G in zip(step.hidden, ref):
+        assert torch.equal(L["G"], G), L["hl"].name
+    # the step is bound to its own input tensors again
+    step.run()
+    torch.cuda.synchronize()
+    for L, G in zip(step.hidden, ref):
+        assert torch.equal(L["G"], G), L["hl"].name
