@@ -526,6 +526,7 @@ def main():
                "noise_ceiling_frac": dominant.get("noise_ceiling_frac")},
             "noise_ceiling": ceiling,
             "kernels": kernels,
+            "layers": layer_report(step, stages),
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches_per_step(step) * args.steps,
@@ -593,6 +594,21 @@ def traffic_bytes(terms, K, T, d_out):
     if not terms or any(u not in counts for _, u in terms):
         return None
     return sum(b * counts[u] for b, u in terms)
+
+
+def layer_report(step, stages):
+    """The metric per layer step: draws x tokens over the layer's own stages (a hidden layer: scan, reduction and
+    weight estimate; the head: logits, its chunk passes and weight estimate), on this rank."""
+    per = {}
+    for name, ms in zip(step.stage_names, stages):
+        layer = name.split(":")[0]
+        per[layer] = per.get(layer, 0.0) + float(ms)
+    out = []
+    for layer, ms in per.items():
+        draws = step.head["draws"] if layer == "head" else step.draws
+        units = draws * step.w.T * (step.head["Vr"] / step.w.V if layer == "head" else 1)
+        out.append({"layer": layer, "ms": ms, "draws_x_tokens_per_s": units / (ms / 1e3) if ms > 0 else None})
+    return out
 
 
 def noise_ceiling(step, K):

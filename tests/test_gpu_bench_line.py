@@ -36,7 +36,7 @@ def test_bench_line_contract(workload, draws):
     line = run_bench("--workload", workload, "--draws", str(draws))
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks",
-                "status", "noise_ceiling", "kernels"):
+                "status", "noise_ceiling", "kernels", "layers"):
         assert key in line, key
     assert line["status"] == "ok"
     assert line["n_gpus"] == 1 and line["steps"] == 2 and line["warmup"] == 3
@@ -47,6 +47,15 @@ def test_bench_line_contract(workload, draws):
     roof = line["roofline"]
     assert roof["bound"] in ("alu", "hbm", "tensor") and 0 < roof["frac"] == pytest.approx(
         roof["achieved"] / roof["peak"])
+    # the metric per layer step: each layer's draws x tokens over its own stages, which add up to the step
+    names = {L["layer"] for L in line["layers"]}
+    assert names == {k["name"].split(":")[0] for k in line["kernels"]}
+    stage_ms = sum(L["ms"] for L in line["layers"])
+    assert stage_ms <= line["ms_per_step"] * 1.001 + 1e-3
+    if workload == "hidden_sweep_bf16":          # not launch-bound: the stages fill the step
+        assert stage_ms == pytest.approx(line["ms_per_step"], rel=0.02)
+    for L in line["layers"]:
+        assert L["draws_x_tokens_per_s"] == pytest.approx(draws * line["config"]["tokens_per_rank"] / (L["ms"] / 1e3))
     ceil = line["noise_ceiling"]
     assert ceil["kernel"] == "noise_sum_kernel" and ceil["gaussians_per_s"] > 0
     alu = [k for k in line["kernels"] if k.get("bound") == "alu"]
