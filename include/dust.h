@@ -206,7 +206,7 @@ size_t dust_layer_estimate_weight_grad_workspace(int draw_count, int T, int d_in
  * [CA, weight equation] G_W[o][i] (+)= sum_t g_hat[t][o] X[t][i].
  * g_hat: [T][d_out] of dtype g_dt, X: [T][d_in] of dtype x_dt.  Both bf16:
  * the tcgen05 tensor cores with fp32 accumulation in TMEM when d_in and d_out
- * are multiples of 16 and the pointers 128-byte aligned (else CUDA cores);
+ * are multiples of 8 (16-byte rows for the TMA; else CUDA cores), any T;
  * both fp32: fp32 CUDA cores; mixed (fp32 g with bf16 X, or bf16 g with fp32
  * X): CUDA cores, each bf16 element widened to fp32 exactly, fp32 products.
  * G_W: [d_out][d_in] fp32 (the layout of W).  Split over T with a fixed-order
@@ -219,7 +219,10 @@ size_t dust_weight_grad_workspace(int T, int d_in, int d_out, dust_dtype g_dt, d
 
 /* ------------------------------------------------------------------ a2: logits
  * Clean head forward Z[t][v] = sum_k X[t][k] W[v][k] (no bias), fp32 out.
- * X: [T][d_in], W: [V][d_in] of dtype dt (bf16: tcgen05; f32: CUDA cores).
+ * X: [T][d_in], W: [V][d_in] of dtype dt (bf16: tcgen05 when d_in is a
+ * multiple of 8, else CUDA cores; f32: CUDA cores).  Z: [T][V] fp32, 16-byte
+ * aligned; written by TMA stores when V is a multiple of 4, by row stores
+ * otherwise (the same values).
  * Workspace: dust_logits_workspace(). */
 dust_status dust_logits(const void *X, const void *W, dust_dtype dt, int T, int d_in,
                         int V, float *Z, void *ws, size_t ws_bytes, void *stream);
