@@ -119,6 +119,20 @@ def test_reward_scan_split_parity(orc, lengths, K, gamma):
     np.testing.assert_array_equal(host(inplace).view(np.uint32), r.view(np.uint32))
 
 
+def test_reward_scan_split_one_very_long_sequence(orc):
+    """The case the chunked scan is timed on: one sequence of 262144 tokens
+    (256 chunks per draw row), K = 16, gamma = 0.99; every reward against the
+    oracle's recurrence, and the per-sequence scan's rewards."""
+    T, K, gamma = 262144, 16, 0.99
+    off = np.array([0, T], np.int32)
+    c = I.normal((K, T), 0.01, seed=2026)
+    ref = orc.reward_scan(c, off, gamma)
+    gc, goff = cu(c), cu(off)
+    r = host(dust.reward_scan_split(gc, goff, gamma))
+    assert rel_err(r, ref) < 1e-5
+    assert rel_err(host(dust.reward_scan(gc, goff, gamma)), ref) < 1e-5
+
+
 def test_layer_estimate_long_sequence_uses_chunked_scan(orc):
     """K x n_seq small and one long sequence: the estimate runs the chunked scan internally."""
     T, K, d = 9000, 4, 16
