@@ -295,7 +295,8 @@ def test_head_step_small_fp32(orc):
     assert rel_err(host(cached["G_W"]), G_ref) < FP32_TOL
 
 
-@pytest.mark.parametrize("sigma", [0.005, 0.02, 0.05])   # the three expm1 tiers of the head kernel
+@pytest.mark.parametrize("sigma", [0.005, 0.02, 0.05, 0.1, 0.3])   # the four expm1 tiers of the head kernel
+                                                                   # (0.05 and 0.1: the x^8 series)
 def test_head_step_chunks_and_split(orc, sigma):
     """Several chunks, draw split with accumulate, target ids on chunk edges."""
     T, V, Vc, K = 40, 768, 256, 10

@@ -64,7 +64,7 @@ def test_estimate_random_shapes(orc, lengths, d_out, K, split, gamma, seed, tb):
 
 @settings(**dict(SETTINGS, max_examples=40))
 @given(T=st.integers(1, 40), n_chunks=st.integers(1, 4), Vc=st.sampled_from([128, 256, 384, 1024]),
-       K=st.integers(1, 6), sigma=st.sampled_from([0.005, 0.02, 0.05]), seed=st.integers(0, 10_000),
+       K=st.integers(1, 6), sigma=st.sampled_from([0.005, 0.02, 0.05, 0.3]), seed=st.integers(0, 10_000),
        first=st.integers(0, 3), tb=st.integers(0, 2**31 - 1000))
 def test_head_random_shapes(orc, T, n_chunks, Vc, K, sigma, seed, first, tb):
     """Head step (cached logits) over a random range of its chunks, with the
